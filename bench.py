@@ -1,0 +1,500 @@
+"""Throughput bench of the bifocal hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * prefill of the Qwen3-8B-shaped layer at 128K (batch 1, 32 q heads / 8 kv
+    heads, head_dim 128, RoPE base 1e6, L 131072, w_pretrained 32768 -> G 4,
+    w0 4096): correction pass + fused tcgen05 attention;
+  * decode of the Qwen3-4B-shaped layer at 128K (32 / 8 heads, head_dim 128,
+    batch 8, cache of 131072 base-rotated keys, G 4, w0 4096).
+`value` is the prefill TFLOP/s (algorithmic 4 * B * Hq * d * L(L+1)/2 per
+step, summed over ranks, divided by the max-over-ranks device time of the
+prefill calls); the decode GB/s (K and V bytes read once) is reported beside
+it.  Inputs are larger than L2 (1 GiB Q, 4 GiB KV cache), so no flush runs
+between steps.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+For N > 1 launch under torch.distributed.run; every rank runs its own
+independent sequences (weak scaling, no data-path collective).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "bifocal prefill TFLOP/s @128K; decode HBM GB/s @128K; % of B200 roofline"
+
+PREFILL = dict(workload="qwen3-8b-shaped bifocal prefill, single layer", B=1, L=131072, Hq=32, Hkv=8, D=128,
+               W=32768, w0=4096, base=1e6)
+DECODE = dict(workload="qwen3-4b-shaped bifocal decode", B=8, L=131072, Hq=32, Hkv=8, D=128, W=32768, w0=4096,
+              base=1e6)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def prefill_flop(c):
+    return 4.0 * c["B"] * c["Hq"] * c["D"] * c["L"] * (c["L"] + 1) / 2.0
+
+
+def decode_bytes(c):
+    return 2.0 * c["B"] * c["L"] * c["Hkv"] * c["D"] * 2.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic():
+    """Per-launch DRAM bytes of the timed kernels from the committed ncu summary,
+    valid only while the kernel sources hash to the value recorded with them."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    try:
+        with open(path) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    cur = sources_hash()
+    return {k: v for k, v in data.items() if isinstance(v, dict) and v.get("sources") == cur}
+
+
+def sources_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rope_context_extension_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def gen_on_device(shape, seed, dev):
+    import torch
+    g = torch.Generator(device=dev).manual_seed(seed)
+    return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    from rope_context_extension_b200 import jetlong as jl
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    P, Dc = PREFILL, DECODE
+    seed = 1000 * rank
+
+    # prefill buffers (resident in HBM)
+    q = gen_on_device((P["B"], P["L"], P["Hq"], P["D"]), seed + 0, dev)
+    k = gen_on_device((P["B"], P["L"], P["Hkv"], P["D"]), seed + 1, dev)
+    v = gen_on_device((P["B"], P["L"], P["Hkv"], P["D"]), seed + 2, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(P["B"], P["Hq"], P["L"], dtype=torch.float32, device=dev)
+    ws = torch.empty(jl.jl_prefill_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]), dtype=torch.uint8,
+                     device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    # decode buffers
+    dq = gen_on_device((Dc["B"], Dc["Hq"], Dc["D"]), seed + 3, dev)
+    kc = gen_on_device((Dc["B"], Dc["L"], Dc["Hkv"], Dc["D"]), seed + 4, dev)
+    vc = gen_on_device((Dc["B"], Dc["L"], Dc["Hkv"], Dc["D"]), seed + 5, dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty(Dc["B"], Dc["Hq"], dtype=torch.float32, device=dev)
+    dws = torch.zeros(jl.jl_decode_workspace_bytes(Dc["B"], Dc["L"], Dc["Hq"], Dc["Hkv"], Dc["D"]),
+                      dtype=torch.uint8, device=dev)
+
+    pkw = dict(w0=P["w0"], w_pretrained=P["W"], stream=stream)
+
+    def prefill_step(evs=None, w0=None):
+        w = P["w0"] if w0 is None else w0
+        if evs:
+            evs[0].record(stream)
+        jl.jl_prefill_correction(q, k, w0=w, w_pretrained=P["W"], rope_base=P["base"], workspace=ws, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        jl.jl_prefill_attention(q, k, v, o, lse, w0=w, w_pretrained=P["W"], workspace=ws, dev_error=err,
+                                stream=stream)
+        if evs:
+            evs[2].record(stream)
+
+    def decode_step(evs=None, w0=None):
+        w = Dc["w0"] if w0 is None else w0
+        if evs:
+            evs[0].record(stream)
+        jl.jl_bifocal_decode(dq, kc, vc, do, dlse, L=Dc["L"], w0=w, w_pretrained=Dc["W"], rope_base=Dc["base"],
+                             workspace=dws, dev_error=err, stream=stream)
+        if evs:
+            evs[1].record(stream)
+
+    for _ in range(args.warmup):
+        prefill_step()
+        decode_step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    dev_ = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(K):
+        prefill_step(pev[i])
+        decode_step(dev_[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError("device pipeline timeout flag set during the timed region")
+
+    total_ms = t0.elapsed_time(t1)
+    corr_ms = sum(e[0].elapsed_time(e[1]) for e in pev) / K
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in pev) / K
+    dec_ms = sum(e[0].elapsed_time(e[1]) for e in dev_) / K
+    pre_ms = corr_ms + attn_ms
+    total_ms = max_over_ranks(total_ms, world)
+    pre_ms_max = max_over_ranks(pre_ms, world)
+    attn_ms_max = max_over_ranks(attn_ms, world)
+    dec_ms_max = max_over_ranks(dec_ms, world)
+
+    flop = prefill_flop(P)
+    dbytes = decode_bytes(Dc)
+    value = world * flop / (pre_ms_max * 1e-3) / 1e12
+    attn_tflops = flop / (attn_ms_max * 1e-3) / 1e12
+    dec_gbs = world * dbytes / (dec_ms_max * 1e-3) / 1e9
+    dec_gbs_kernel = dbytes / (dec_ms_max * 1e-3) / 1e9
+
+    # plain causal RoPE from the same kernels (w0 = L), measured after the timed region
+    def time_calls(fn, reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    plain_pre_ms = time_calls(lambda: prefill_step(w0=P["L"]), max(2, K // 2))
+    plain_dec_ms = time_calls(lambda: decode_step(w0=Dc["L"]), max(2, K // 2))
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h_bytes = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+        d_bytes = ho.numel() * 2
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(2, K // 2)
+        torch.cuda.synchronize()
+        barrier(world)
+        a.record(stream)
+        for _ in range(reps):
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            jl.jl_bifocal_prefill(q, k, v, o, lse, w0=P["w0"], w_pretrained=P["W"], rope_base=P["base"],
+                                  workspace=ws, dev_error=err, stream=stream)
+            ho.copy_(o, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / reps, world)
+        e2e = {"value": round(world * flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h_bytes), "d2h_bytes_per_step": int(d_bytes),
+               "ms_per_step": round(e2e_ms, 3), "api": "jl_bifocal_prefill"}
+
+    peaks, peak_kind = load_peaks()
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    traffic = load_traffic()
+    out = None
+    if rank == 0:
+        cpu = None if args.no_cpu_baseline else cpu_baseline_sample(seconds=args.cpu_seconds)
+        out = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": round(total_ms / K, 3),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded randn on device, N(0,1) bf16; inputs larger than L2, no flush)",
+            "config": {
+                "workload": P["workload"] + " + " + Dc["workload"],
+                "prefill": {k_: P[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")},
+                "decode": {k_: Dc[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")},
+                "query_shift": "self_extend",
+                "l2": "inputs larger than L2",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            },
+            "prefill": {"ms": round(pre_ms_max, 3), "correction_ms": round(corr_ms, 3),
+                        "attention_ms": round(attn_ms_max, 3), "tokens_per_s": round(world * P["L"] * P["B"] /
+                                                                                     (pre_ms_max * 1e-3), 1),
+                        "attention_tflops": round(attn_tflops, 2)},
+            "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "ms": round(dec_ms_max, 4),
+                       "tokens_per_s": round(world * Dc["B"] / (dec_ms_max * 1e-3), 1),
+                       "roofline": {"bound": "hbm", "achieved": round(dec_gbs_kernel, 1),
+                                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": round(dec_gbs_kernel / peaks["hbm_gbs"], 4),
+                                    "traffic": traffic.get("decode", {}).get("bytes_per_launch"),
+                                    "peak_source": f"{peak_kind} hbm_gbs"}},
+            "plain_rope_same_kernels": {
+                "prefill_ms": round(plain_pre_ms, 3),
+                "prefill_tflops": round(flop / (plain_pre_ms * 1e-3) / 1e12, 2),
+                "decode_ms": round(plain_dec_ms, 4),
+                "decode_gbs": round(dbytes / (plain_dec_ms * 1e-3) / 1e9, 1),
+            },
+            "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": tensor_peak,
+                         "unit": "TFLOP/s", "frac": round(attn_tflops / tensor_peak, 4),
+                         "traffic": traffic.get("prefill_attention", {}).get("bytes_per_launch"),
+                         "kernel": "bifocal_prefill_kernel<128>",
+                         "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a multi-second loop)"},
+            "e2e": e2e,
+            "gpu_launches": K * 4,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return out
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_rows_timed(n_rows, seed=0):
+    """Time the fp64 oracle on n_rows query rows (all of one KV head's query
+    heads) of the 128K prefill workload; returns (algorithmic flop, seconds)."""
+    import numpy as np
+    import torch
+    from oracle import jetlong_oracle as jo
+    P = PREFILL
+    g = torch.Generator("cpu").manual_seed(seed)
+    r = P["Hq"] // P["Hkv"]
+    kk = torch.randn(P["L"], P["D"], generator=g).to(torch.bfloat16).double().numpy()
+    vv = torch.randn(P["L"], P["D"], generator=g).to(torch.bfloat16).double().numpy()
+    qq = torch.randn(r, n_rows, P["D"], generator=g).to(torch.bfloat16).double().numpy()
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(P["L"], size=n_rows, replace=False))
+    p = jo.BifocalParams(L=P["L"], w0=P["w0"], w_pretrained=P["W"], base=P["base"])
+    t = time.perf_counter()
+    for h in range(r):
+        jo.attention_rows(qq[h], rows, kk, vv, p)
+    dt = time.perf_counter() - t
+    flop = 4.0 * P["D"] * float(np.sum(rows + 1)) * r
+    return flop, dt, rows
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_sample(seconds=15.0):
+    n = 8
+    flop, dt, _ = _oracle_rows_timed(n)
+    if dt < seconds / 4:
+        n = int(max(8, min(512, n * seconds / max(dt, 1e-3) * 0.8)))
+        flop, dt, _ = _oracle_rows_timed(n, seed=1)
+    return {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"fp64 oracle, {n} random query rows x 4 q heads of one KV head of the 128K prefill "
+                      f"workload, {dt:.1f} s; TFLOP/s from the algorithmic flop of those rows"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        _oracle_rows_timed(2, seed=7)
+    times, flops = [], []
+    for i in range(args.steps):
+        f, dt, _ = _oracle_rows_timed(args.ref_rows, seed=100 + i)
+        flops.append(f)
+        times.append(dt)
+    total = sum(times)
+    value = sum(flops) / total / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded randn, N(0,1) bf16 widened to fp64)",
+        "config": {"workload": PREFILL["workload"],
+                   "prefill": {k_: PREFILL[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")}},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                         "sample": f"each step: {args.ref_rows} random query rows x 4 q heads of one KV head of "
+                                   f"the 128K prefill workload on the fp64 CPU oracle"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--prefill-len", type=int, default=None, help="smaller prefill L (profiling runs only)")
+    ap.add_argument("--decode-len", type=int, default=None, help="smaller decode L (profiling runs only)")
+    ap.add_argument("--decode-batch", type=int, default=None, help="decode batch (default 8)")
+    args = ap.parse_args()
+    if args.prefill_len:
+        PREFILL["L"] = args.prefill_len
+        PREFILL["workload"] += f" (L={args.prefill_len}, profiling size)"
+    if args.decode_len:
+        DECODE["L"] = args.decode_len
+        DECODE["workload"] += f" (L={args.decode_len}, profiling size)"
+    if args.decode_batch:
+        DECODE["B"] = args.decode_batch
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        out = run_reference(args)
+    else:
+        out = run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

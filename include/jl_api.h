@@ -1,0 +1,163 @@
+/*
+ * jl_api.h -- C ABI of the B200 (sm_100a) Dynamic Bifocal RoPE attention
+ * library (libjetlong.so).
+ *
+ * The method (Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal
+ * RoPE; Jet-Long review (romaanj.github.io), "Method"; gist.science technical
+ * summary, "Methodologie §1-§2"):
+ *   G     = max(1, ceil(L / w_pretrained)), from the current length L
+ *   f(x)  = floor(x / G)                    remote position map
+ *   a causal pair (query i, key j) with i - j < w0 keeps its base RoPE score;
+ *   every other causal pair is scored with the query at p_q(i) and the key at
+ *   f(j).  Keys stay in the cache rotated at their absolute positions; the
+ *   correction rotations R(p_q(i) - i) and R(f(j) - j) are applied on the fly.
+ *
+ * The pages leave the query-side remote position unstated.  `mode` selects it:
+ *   JL_QSHIFT_SELF_EXTEND  p_q(i) = floor(i/G) + (w0 - floor(w0/G))
+ *                          (remote distances continue from w0; default)
+ *   JL_QSHIFT_NONE         p_q(i) = floor(i/G)
+ * Both reduce to base RoPE at G = 1.
+ *
+ * Conventions shared by every entry point:
+ *   - bf16 tensors are row-major and contiguous:
+ *       Q, O (prefill) [B, L, Hq, D]; K, V (prefill) [B, L, Hkv, D];
+ *       KV cache (decode) [B, Lmax, Hkv, D]; q, o (decode) [B, Hq, D];
+ *       LSE fp32: prefill [B, Hq, L], decode [B, Hq] (natural log of the sum
+ *       of exp of the scaled scores).
+ *   - Q and K hold rows already rotated at their absolute (base) positions with
+ *     half-split RoPE pairs (t, t + D/2), theta_t = rope_base^(-2t/D).
+ *   - D (head_dim) is 64 or 128; Hq % Hkv == 0; 1 <= L; w0 >= 0;
+ *     w_pretrained >= 1.  softmax_scale == 0 means 1/sqrt(D).
+ *   - Device pointers must be 16-byte aligned.  The caller owns every buffer
+ *     (inputs, outputs and scratch); the library never allocates device
+ *     memory and never writes its inputs.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = default
+ *     stream).  The return value reports argument checks and launch errors.
+ *     Device-side failures (a pipeline wait that ran out of time) are written
+ *     to *dev_error (a device int, may be NULL) as a non-zero value; the
+ *     outputs are then invalid.
+ *   - Reentrant; no global state beyond cached kernel attributes.
+ */
+#ifndef JL_API_H
+#define JL_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  JL_OK = 0,
+  JL_ERR_INVALID_ARG = -1,    /* null pointer, bad size or range */
+  JL_ERR_UNSUPPORTED = -2,    /* shape the kernels do not handle (e.g. D not 64/128) */
+  JL_ERR_ALIGNMENT = -3,      /* a device pointer is not 16-byte aligned */
+  JL_ERR_WORKSPACE = -4,      /* scratch missing or smaller than required */
+  JL_ERR_CUDA = -5,           /* a CUDA runtime / driver call failed */
+  JL_ERR_DEVICE_TIMEOUT = -6  /* reserved: host-side report of a device timeout */
+} jl_status;
+
+typedef enum { JL_QSHIFT_NONE = 0, JL_QSHIFT_SELF_EXTEND = 1 } jl_qshift;
+
+/* Human-readable name of a status code (static string). */
+const char* jl_status_string(int status);
+
+/*
+ * Group size G = max(1, ceil(L / w_pretrained)) (Jet-Long review, "Method";
+ * gist.science summary, "Methodologie §1").  Host only.
+ * Errors: JL_ERR_INVALID_ARG if L < 0, w_pretrained < 1 or G_out is NULL.
+ */
+int jl_group_size(int64_t L, int64_t w_pretrained, int64_t* G_out);
+
+/*
+ * Remote positions for a length-L sequence (host arrays of L int32 each, either
+ * may be NULL): q_pos_out[i] = p_q(i) (see `mode`), k_pos_out[j] = f(j).
+ * Host only; used to check the position maps bit-exactly.
+ * Errors: JL_ERR_INVALID_ARG for L < 1, w0 < 0, w_pretrained < 1, a bad mode,
+ * or positions that do not fit int32.
+ */
+int jl_remote_positions(int64_t L, int64_t w0, int64_t w_pretrained, int mode, int32_t* q_pos_out,
+                        int32_t* k_pos_out);
+
+/*
+ * Scratch bytes jl_bifocal_prefill needs: space for the remote-rotated Q and K
+ * rows (2 * B * L * (Hq + Hkv) * D bytes plus alignment).  0 on bad arguments.
+ */
+size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim);
+
+/*
+ * Fused bifocal causal prefill (self-attention of L new tokens).
+ *   q [B, L, Hq, D], k / v [B, L, Hkv, D]: bf16 device, base-rotated, read only.
+ *   o [B, L, Hq, D] bf16 device (written); lse [B, Hq, L] fp32 device or NULL.
+ *   w0: band width of exact base-RoPE scoring (i - j < w0); w0 >= L, or
+ *   L <= w_pretrained (G = 1), gives plain causal RoPE attention.
+ *   workspace: device scratch of at least jl_prefill_workspace_bytes(...) bytes
+ *   (contents on entry do not matter; overwritten).
+ * Launches: jl_prefill_correction (one correction-rotation kernel for Q and one
+ * for K, skipped when every pair is local), then jl_prefill_attention (the
+ * fused tcgen05 attention kernel).
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_ALIGNMENT,
+ * JL_ERR_WORKSPACE, JL_ERR_CUDA; nothing is launched on an argument error.
+ */
+int jl_bifocal_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L,
+                       int Hq, int Hkv, int head_dim, int w0, int w_pretrained, double rope_base,
+                       float softmax_scale, int mode, void* workspace, size_t workspace_bytes,
+                       int* dev_error, void* stream);
+
+/*
+ * First stage of jl_bifocal_prefill, exposed so the two stages can be timed or
+ * scheduled separately: writes the correction-rotated rows to `workspace`
+ * (fp16, [B, L, Hq, D] for R(p_q(i) - i) Q_i followed by [B, L, Hkv, D] for
+ * R(f(j) - j) K_j, the second at offset round_up(2 * B * L * Hq * D, 256)).
+ * Only rows that have a remote partner are written (queries i >= w0, keys
+ * j < L - w0).  The correction identity is the additive composition of RoPE
+ * rotations (gist.science summary, "§2 On-the-Fly Correctie Rotatie").
+ * Launches nothing when every pair is local.  Errors as jl_bifocal_prefill.
+ */
+int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, int Hkv, int head_dim, int w0,
+                          int w_pretrained, double rope_base, int mode, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * Second stage of jl_bifocal_prefill: the fused tcgen05 attention kernel
+ * (one launch), reading Q, K, V and the corrected rows that
+ * jl_prefill_correction left in `workspace` (same w0 / w_pretrained / mode).
+ * Errors as jl_bifocal_prefill.
+ */
+int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
+                         int Hkv, int head_dim, int w0, int w_pretrained, float softmax_scale, int mode,
+                         const void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
+
+/*
+ * Scratch bytes jl_bifocal_decode needs on this device (split partials and one
+ * ticket counter per (batch, KV head)).  0 on bad arguments.
+ */
+size_t jl_decode_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim);
+
+/*
+ * Fused bifocal decode: one new query token per sequence at position L - 1
+ * against the first L cache entries (L counts the new token's own key).
+ *   q [B, Hq, D] bf16 device, rotated at position L - 1.
+ *   k_cache / v_cache [B, cache_len, Hkv, D] bf16 device, keys rotated at their
+ *   absolute positions; read only, never rewritten; L <= cache_len.
+ *   o [B, Hq, D] bf16 device; lse [B, Hq] fp32 device or NULL.
+ *   Hq / Hkv <= 8.
+ *   workspace: device scratch of at least jl_decode_workspace_bytes(...) bytes.
+ *   Its ticket counters must be zero before the first call (allocate it
+ *   zero-filled); every call leaves them at zero again.  Calls that share a
+ *   workspace must not overlap on the GPU.
+ * Launches one kernel.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_ALIGNMENT,
+ * JL_ERR_WORKSPACE, JL_ERR_CUDA; nothing is launched on an argument error.
+ */
+int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                      float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
+                      double rope_base, float softmax_scale, int mode, void* workspace,
+                      size_t workspace_bytes, int* dev_error, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JL_API_H */

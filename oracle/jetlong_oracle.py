@@ -47,6 +47,7 @@ forms a correction rotation.  Library primitives used as steps: ``numpy``
 
 from __future__ import annotations
 
+import hashlib
 import math
 from dataclasses import dataclass
 
@@ -134,6 +135,27 @@ def rope_frequencies(d: int, base: float) -> np.ndarray:
     return np.power(np.float64(base), -2.0 * t / d)
 
 
+_CS_CACHE: dict = {}
+
+
+def _cos_sin(pos, d: int, base: float):
+    """cos / sin of pos * theta_t (fp64), memoised on the position values."""
+    pos = np.asarray(pos, dtype=np.float64)
+    key = None
+    if pos.size >= 4096:
+        key = (pos.shape, d, float(base), hashlib.blake2b(pos.tobytes(), digest_size=16).digest())
+        hit = _CS_CACHE.get(key)
+        if hit is not None:
+            return hit
+    ang = pos[..., None] * rope_frequencies(d, base)
+    out = (np.cos(ang), np.sin(ang))
+    if key is not None:
+        if len(_CS_CACHE) > 16:
+            _CS_CACHE.clear()
+        _CS_CACHE[key] = out
+    return out
+
+
 def rope_rotate(x: np.ndarray, pos, base: float) -> np.ndarray:
     """Rotate rows of x (..., d) to integer positions ``pos`` (broadcast on ...).
 
@@ -144,8 +166,7 @@ def rope_rotate(x: np.ndarray, pos, base: float) -> np.ndarray:
     x = np.asarray(x, dtype=np.float64)
     d = x.shape[-1]
     h = d // 2
-    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_frequencies(d, base)
-    c, s = np.cos(ang), np.sin(ang)
+    c, s = _cos_sin(pos, d, base)
     lo, hi = x[..., :h], x[..., h:]
     return np.concatenate([lo * c - hi * s, hi * c + lo * s], axis=-1)
 
@@ -167,12 +188,22 @@ class BifocalParams:
         return 1.0 / math.sqrt(d) if not self.scale else float(self.scale)
 
 
+def rotated_keys(k: np.ndarray, p: BifocalParams):
+    """(R(j) k_raw_j, R(f(j)) k_raw_j) for base-rotated keys k (L, d), fp64."""
+    k = np.asarray(k, dtype=np.float64)
+    G = group_size(p.L, p.w_pretrained)
+    j = np.arange(k.shape[0], dtype=np.int64)
+    k_hat = rope_rotate(k, -j, p.base)               # raw key vectors
+    return rope_rotate(k_hat, j, p.base), rope_rotate(k_hat, key_remote_position(j, G), p.base)
+
+
 def bifocal_scores(q_rows: np.ndarray, q_pos: np.ndarray, k: np.ndarray,
-                   p: BifocalParams) -> np.ndarray:
+                   p: BifocalParams, keys=None) -> np.ndarray:
     """Scaled bifocal scores for query rows against keys 0..L-1 (fp64).
 
     q_rows: (n, d) base-rotated queries at absolute positions q_pos (n,).
     k:      (L, d) base-rotated keys at positions 0..L-1.
+    keys:   optional ``rotated_keys(k, p)`` (the same values, computed once).
     Returns (n, L) with -inf on non-causal pairs (j > i).
     """
     n, d = q_rows.shape
@@ -180,12 +211,10 @@ def bifocal_scores(q_rows: np.ndarray, q_pos: np.ndarray, k: np.ndarray,
     G = group_size(p.L, p.w_pretrained)
     j = np.arange(L, dtype=np.int64)
     i = np.asarray(q_pos, dtype=np.int64)
+    k_loc, k_rem = rotated_keys(k, p) if keys is None else (keys[0][:L], keys[1][:L])
     q_hat = rope_rotate(q_rows, -i, p.base)          # raw query vectors
-    k_hat = rope_rotate(k, -j, p.base)               # raw key vectors
     q_loc = rope_rotate(q_hat, i, p.base)
-    k_loc = rope_rotate(k_hat, j, p.base)
     q_rem = rope_rotate(q_hat, query_remote_position(i, G, p.w0, p.mode), p.base)
-    k_rem = rope_rotate(k_hat, key_remote_position(j, G), p.base)
     s_loc = q_loc @ k_loc.T
     s_rem = q_rem @ k_rem.T
     local = is_local(i[:, None], j[None, :], p.w0)
@@ -210,11 +239,13 @@ def attention_rows(q_rows, q_pos, k, v, p: BifocalParams, chunk: int = 64):
     q_pos = np.asarray(q_pos, dtype=np.int64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
+    kmax_all = int(q_pos.max()) + 1
+    keys = rotated_keys(k[:kmax_all], p)
     outs, lses = [], []
     for a in range(0, q_rows.shape[0], chunk):
         qp = q_pos[a:a + chunk]
         kmax = int(qp.max()) + 1                      # keys beyond the last row are masked
-        s = bifocal_scores(q_rows[a:a + chunk], qp, k[:kmax], p)
+        s = bifocal_scores(q_rows[a:a + chunk], qp, k[:kmax], p, keys=keys)
         o, lse = softmax_rows(s, v[:kmax])
         outs.append(o)
         lses.append(lse)

@@ -1,0 +1,503 @@
+// Fused Dynamic Bifocal RoPE decode for sm_100a: one new query token per
+// sequence (at position L - 1) against a cache of base-rotated keys.
+//
+// The cache holds keys rotated at their absolute positions and is never
+// rewritten (Jet-Long review, "Method"; gist.science summary, "§2 On-the-Fly
+// Correctie Rotatie").  Keys with (L - 1) - j < w0 are scored with the query as
+// given; every other key is scored with the correction rotations applied in
+// registers: the query is rotated by dq = p_q(L-1) - (L-1) and key j by
+// dk(j) = f(j) - j.
+//
+// Split-KV layout: grid (splits, Hkv, B); each CTA streams a contiguous run of
+// 64-key tiles of one KV head through a 3-stage TMA ring (128-byte swizzled so
+// ldmatrix is conflict-free) and scores all r = Hq / Hkv query heads of that KV
+// head at once with mma.sync m16n8k16 (heads on the M axis, 16 keys per warp).
+//
+// Correction rotation of keys, per warp tile of 16 keys starting at j0:
+//   dk(j) = dk(j0) - e(j) with e(j) in [0, 15]; the query side carries
+//   R(dq - dk(j0)) q (kept in fp32, advanced by one fixed small rotation per
+//   tile), and the key side only needs R(-e(j)) from a 16-row table, applied
+//   to the key fragments in registers before the product.  Every angle with a
+//   large argument is formed and reduced in fp64 once per CTA.  Corrected
+//   operands enter the products as bf16 hi + lo pairs, so the remote scores
+//   carry about 16 significant bits, like the unrotated local ones.
+//
+// Partials (running max, sum, unnormalised O) go to caller scratch; the last
+// CTA of each (batch, KV head) - found with an atomic ticket, no spinning -
+// merges them with a warp-shuffle log-sum-exp combine.
+#include "jl_kernels.cuh"
+
+namespace jl {
+
+namespace {
+
+constexpr int kDecKeys = 64;   // keys per stage
+constexpr int kDecStages = 3;
+constexpr int kDecThreads = 160;  // 4 consumer warps + 1 TMA warp
+constexpr int kMaxR = 8;       // query heads per KV head handled (M rows used)
+
+template <int D>
+struct DecCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kDecKeys * D * 2;  // one of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kERow = (D / 2 + 8) * 8;        // bytes per E row (padded)
+  static constexpr int kEOff = kDecStages * kStageBytes;
+  static constexpr int kFOff = kEOff + 16 * kERow;
+  static constexpr int kQ0Off = kFOff + 2 * (D / 2) * 8;  // [4 warps][D/2] initial query factors
+  static constexpr int kBarOff = kQ0Off + 4 * (D / 2) * 8;
+  static constexpr int kSmem = kBarOff + 128 + 1024;
+  static constexpr int kNT = D / 8;                    // t values per lane
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// (a, b) -> bf16x2 hi = round(a, b) and lo = round(a - hi_a, b - hi_b).
+__device__ __forceinline__ void split_pair_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  lo = pack_bf16x2(a - bf16lo_to_f32(hi), b - bf16hi_to_f32(hi));
+}
+
+// Rotate the bf16 pairs (x, y) (two lanes of a bf16x2 word each) by the complex
+// factors (c0, s0), (c1, s1) and return the results as hi / lo bf16 parts.
+__device__ __forceinline__ void rot_split_bf16(uint32_t xw, uint32_t yw, float c0, float s0, float c1, float s1,
+                                               uint32_t& xh, uint32_t& xl, uint32_t& yh, uint32_t& yl) {
+  const float x0 = bf16lo_to_f32(xw), x1 = bf16hi_to_f32(xw);
+  const float y0 = bf16lo_to_f32(yw), y1 = bf16hi_to_f32(yw);
+  split_pair_bf16(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1, xh, xl);
+  split_pair_bf16(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1, yh, yl);
+}
+
+__device__ __forceinline__ void named_sync_consumers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int D>
+__global__ void __maxnreg__(200)
+    bifocal_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ DecodeArgs args) {
+  using C = DecCfg<D>;
+  constexpr int H2 = D / 2;
+  constexpr int KS = D / 16;   // k-steps of the score product
+  constexpr int KS2 = D / 32;  // k-steps holding the first half of each pair
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 64);
+  volatile int* ticket_slot = reinterpret_cast<volatile int*>(smem + C::kBarOff + 68);
+  auto full_bar = [&](int s) -> uint32_t { return smem_addr(&bars[s]); };
+  auto empty_bar = [&](int s) -> uint32_t { return smem_addr(&bars[kDecStages + s]); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int r = args.r;
+  const int L = args.L;
+  const int t_begin = (int)(((int64_t)split * args.ntiles) / args.splits);
+  const int t_end = (int)(((int64_t)(split + 1) * args.ntiles) / args.splits);
+  const int ntile = t_end - t_begin;
+  const int G = (int)args.G;
+  const bool all_local = args.all_local != 0;
+  const int local_from = all_local ? 0 : L - args.w0;  // keys j >= local_from are local
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 4);
+    }
+    fence_mbar_init();
+  }
+  // Correction tables (consumers only use them; everyone helps fill them):
+  //   E[e][t]  rotation by -e (e in [0, 16)) applied to keys within a warp tile
+  //   F[k][t]  advance of the query factor from one warp tile to the next
+  //            (64 keys later), k = (number of new groups) - floor(64 / G)
+  //   Q0[w][t] rotation by dq - dk(j0) for warp w's first tile
+  float2* E = reinterpret_cast<float2*>(smem + C::kEOff);
+  float2* F = reinterpret_cast<float2*>(smem + C::kFOff);
+  float2* Q0 = reinterpret_cast<float2*>(smem + C::kQ0Off);
+  if (!all_local) {
+    const int q64 = 64 / G;
+    for (int idx = threadIdx.x; idx < 22 * H2; idx += blockDim.x) {
+      const int row = idx / H2, t = idx % H2;
+      double turns;
+      if (row < 16) {
+        turns = -(double)row;
+      } else if (row < 18) {
+        turns = -(double)(q64 + (row - 16) - 64);  // -(dk(j0 + 64) - dk(j0))
+      } else {
+        const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18);
+        turns = (double)(args.dq - (j0 / G - j0));
+      }
+      double sn, cs;
+      sincos(turns * args.theta[t], &sn, &cs);
+      const float2 v = make_float2((float)cs, (float)sn);
+      if (row < 16)
+        E[row * (C::kERow / 8) + t] = v;
+      else if (row < 18)
+        F[(row - 16) * H2 + t] = v;
+      else
+        Q0[(row - 18) * H2 + t] = v;
+    }
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      int last = -1;
+      bool ok = true;
+      for (int i = 0; i < ntile; ++i) {
+        const int s = i % kDecStages;
+        const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
+        if (!(ok = mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, args.dev_error))) break;
+        const int key0 = (t_begin + i) * kDecKeys;
+        mbar_arrive_expect_tx(full_bar(s), (uint32_t)C::kStageBytes);
+        const uint32_t st = sbase + s * C::kStageBytes;
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_4d(st + c * (kDecKeys * 128), &tm_k, full_bar(s), c * 64, g, key0, b);
+          tma_load_4d(st + C::kTileBytes + c * (kDecKeys * 128), &tm_v, full_bar(s), c * 64, g, key0, b);
+        }
+        last = i;
+      }
+      if (!ok) {
+        for (int i = max(0, last - kDecStages + 1); i <= last; ++i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(full_bar(i % kDecStages), (uint32_t)(i / kDecStages) & 1u))
+            if (global_timer_ns() - t0 > 100000000ull) break;
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int c4 = lane & 3;        // column group of the mma fragments
+  const int hrow = lane >> 2;     // query head (M row) of this lane
+  const bool head_ok = hrow < r;
+  const int hq = g * r + hrow;
+
+  // Base query A fragments (bf16 as given) and the fp32 query copy in the
+  // lane's t-set: t = 16 ks + 2 c4 + {0, 1, 8, 9}, ks < D/32.
+  uint32_t qa_base[KS][2];
+  float qre[C::kNT], qim[C::kNT];
+  {
+    const __nv_bfloat16* qp = args.q + ((size_t)b * args.Hq + (head_ok ? hq : 0)) * D;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const uint32_t w0v = head_ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks + 2 * c4) : 0u;
+      const uint32_t w2v = head_ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks + 8 + 2 * c4) : 0u;
+      qa_base[ks][0] = w0v;
+      qa_base[ks][1] = w2v;
+    }
+#pragma unroll
+    for (int ks = 0; ks < KS2; ++ks) {
+      qre[4 * ks + 0] = bf16lo_to_f32(qa_base[ks][0]);
+      qre[4 * ks + 1] = bf16hi_to_f32(qa_base[ks][0]);
+      qre[4 * ks + 2] = bf16lo_to_f32(qa_base[ks][1]);
+      qre[4 * ks + 3] = bf16hi_to_f32(qa_base[ks][1]);
+      qim[4 * ks + 0] = bf16lo_to_f32(qa_base[ks + KS2][0]);
+      qim[4 * ks + 1] = bf16hi_to_f32(qa_base[ks + KS2][0]);
+      qim[4 * ks + 2] = bf16lo_to_f32(qa_base[ks + KS2][1]);
+      qim[4 * ks + 3] = bf16hi_to_f32(qa_base[ks + KS2][1]);
+    }
+  }
+  // q^c = R(dq - dk(j0)) q for this warp's first 16-key tile.
+  if (!all_local) {
+#pragma unroll
+    for (int e = 0; e < C::kNT; ++e) {
+      const int t = 16 * (e >> 2) + 2 * c4 + (e & 1) + ((e & 2) ? 8 : 0);
+      const float2 f = Q0[warp * H2 + t];
+      const float x = qre[e], y = qim[e];
+      qre[e] = x * f.x - y * f.y;
+      qim[e] = y * f.x + x * f.y;
+    }
+  }
+
+  float oacc[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+  float m_used = -INFINITY, l_part = 0.f;
+  const float sl2 = args.scale_log2;
+  bool ok = true;
+
+  for (int i = 0; i < ntile; ++i) {
+    const int s = i % kDecStages;
+    const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
+    const int j0 = (t_begin + i) * kDecKeys + 16 * warp;
+
+    // advance q^c from the previous tile's j0 to this one
+    if (!all_local && i > 0) {
+      const int jp = j0 - kDecKeys;
+      const int fidx = ((j0 / G) - (jp / G)) - 64 / G;  // 0 or 1
+      const float2* Fr = F + fidx * H2;
+#pragma unroll
+      for (int e = 0; e < C::kNT; ++e) {
+        const int t = 16 * (e >> 2) + 2 * c4 + (e & 1) + ((e & 2) ? 8 : 0);
+        const float2 f = Fr[t];
+        const float x = qre[e], y = qim[e];
+        qre[e] = x * f.x - y * f.y;
+        qim[e] = y * f.x + x * f.y;
+      }
+    }
+
+    ok = mbar_wait(full_bar(s), ph, abort_flag, args.dev_error);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+
+    if (j0 < L) {
+      const uint32_t kst = sbase + s * C::kStageBytes;
+      const uint32_t vst = kst + C::kTileBytes;
+      // class of this 16-key tile
+      const bool t_local = all_local || j0 >= local_from;
+      const bool t_remote = !all_local && (j0 + 15 < local_from);
+
+      float sacc[2][4];
+      float sloc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sacc[nt][k] = sloc[nt][k] = 0.f;
+
+      // correction rows of this lane's two keys (one per 8-key n-tile)
+      const float4* Er[2];
+      if (!t_local) {
+        const int dk0 = (j0 / G) - j0;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int jn = j0 + 8 * nt + (lane >> 2);
+          const int e = dk0 - ((jn / G) - jn);  // 0..15
+          Er[nt] = reinterpret_cast<const float4*>(E + e * (C::kERow / 8));
+        }
+      }
+
+      // Key fragments are loaded a pair of k-steps at a time: k-step kp holds
+      // the first coordinate of RoPE pairs t in [16kp, 16kp + 16) and k-step
+      // kp + D/32 the second, so each pair is complete in registers.
+#pragma unroll
+      for (int kp = 0; kp < KS2; ++kp) {
+        uint32_t klo[4], khi[4];
+        {
+          const int mi = lane >> 3;
+          const int kr = 16 * warp + (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int ks = kp + hf * KS2;
+            const int u = 2 * (ks & 3) + (mi & 1);
+            const uint32_t addr = kst + (ks >> 2) * (kDecKeys * 128) + kr * 128 + ((u ^ (kr & 7)) << 4);
+            if (hf == 0)
+              ldsm_x4(addr, klo[0], klo[1], klo[2], klo[3]);
+            else
+              ldsm_x4(addr, khi[0], khi[1], khi[2], khi[3]);
+          }
+        }
+        if (!t_remote) {  // local or straddling: base query, keys as stored
+          const uint32_t alo[4] = {qa_base[kp][0], 0u, qa_base[kp][1], 0u};
+          const uint32_t ahi[4] = {qa_base[kp + KS2][0], 0u, qa_base[kp + KS2][1], 0u};
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            mma_bf16(sloc[nt], alo, klo[2 * nt], klo[2 * nt + 1]);
+            mma_bf16(sloc[nt], ahi, khi[2 * nt], khi[2 * nt + 1]);
+          }
+        }
+        if (!t_local) {  // remote or straddling: corrected query and keys
+          // The corrected operands are carried as bf16 hi + lo pairs (about 16
+          // significant bits): the query's hi part sits in M rows 0-7 and its
+          // lo part in rows 8-15 (unused by the r <= 8 heads), so two products
+          // per k-step (keys hi, keys lo) give (q_hi + q_lo) . (k_hi + k_lo)
+          // once rows h and h + 8 are added.
+          uint32_t kah[4], kal[4], kbh[4], kbl[4];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const float4 f01 = Er[nt][(16 * kp + 2 * c4) >> 1];
+            const float4 f23 = Er[nt][(16 * kp + 8 + 2 * c4) >> 1];
+            rot_split_bf16(klo[2 * nt], khi[2 * nt], f01.x, f01.y, f01.z, f01.w, kah[2 * nt], kal[2 * nt],
+                           kbh[2 * nt], kbl[2 * nt]);
+            rot_split_bf16(klo[2 * nt + 1], khi[2 * nt + 1], f23.x, f23.y, f23.z, f23.w, kah[2 * nt + 1],
+                           kal[2 * nt + 1], kbh[2 * nt + 1], kbl[2 * nt + 1]);
+          }
+          uint32_t alo[4], ahi[4];
+          split_pair_bf16(qre[4 * kp + 0], qre[4 * kp + 1], alo[0], alo[1]);
+          split_pair_bf16(qre[4 * kp + 2], qre[4 * kp + 3], alo[2], alo[3]);
+          split_pair_bf16(qim[4 * kp + 0], qim[4 * kp + 1], ahi[0], ahi[1]);
+          split_pair_bf16(qim[4 * kp + 2], qim[4 * kp + 3], ahi[2], ahi[3]);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            mma_bf16(sacc[nt], alo, kah[2 * nt], kah[2 * nt + 1]);
+            mma_bf16(sacc[nt], alo, kal[2 * nt], kal[2 * nt + 1]);
+            mma_bf16(sacc[nt], ahi, kbh[2 * nt], kbh[2 * nt + 1]);
+            mma_bf16(sacc[nt], ahi, kbl[2 * nt], kbl[2 * nt + 1]);
+          }
+        }
+      }
+
+      // scores in log2 units with band selection and the tail mask
+      float x[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int j = j0 + 8 * nt + 2 * c4 + k;
+          const bool loc = all_local || j >= local_from;
+          float v = (loc ? sloc[nt][k] : sacc[nt][k] + sacc[nt][k + 2]) * sl2;
+          if (j >= L) v = -INFINITY;
+          x[nt][k] = v;
+        }
+      float mt = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+      const float m_new = fmaxf(m_used, mt);
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_new > m_used + 8.f) {
+        alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
+        resc = m_used != -INFINITY;
+        l_part *= alpha;
+        m_used = m_new;
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          oacc[n][0] *= alpha;
+          oacc[n][1] *= alpha;
+        }
+      }
+      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+      float p[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          p[nt][k] = ex2_approx(x[nt][k] - msub);
+          l_part += p[nt][k];
+        }
+      const uint32_t pa[4] = {pack_bf16x2(p[0][0], p[0][1]), 0u, pack_bf16x2(p[1][0], p[1][1]), 0u};
+#pragma unroll
+      for (int np = 0; np < D / 16; ++np) {
+        const int mi = lane >> 3;
+        const int kr = 16 * warp + (mi & 1) * 8 + (lane & 7);
+        const int u = 2 * (np & 3) + (mi >> 1);
+        const uint32_t addr = vst + (np >> 2) * (kDecKeys * 128) + kr * 128 + ((u ^ (kr & 7)) << 4);
+        uint32_t v0, v1, v2, v3;
+        ldsm_x4_t(addr, v0, v1, v2, v3);
+        mma_bf16(oacc[2 * np], pa, v0, v1);
+        mma_bf16(oacc[2 * np + 1], pa, v2, v3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(s));
+  }
+
+  // ---------------------------------------------------------- CTA merge
+  l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
+  l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+  named_sync_consumers();  // every warp is done with the stage buffers
+  float* mw = reinterpret_cast<float*>(smem);                    // [4][kMaxR]
+  float* lw = mw + 4 * kMaxR;                                    // [4][kMaxR]
+  float* ow = lw + 4 * kMaxR;                                    // [4][kMaxR][D]
+  if (head_ok) {
+    if (c4 == 0) {
+      mw[warp * kMaxR + hrow] = m_used;
+      lw[warp * kMaxR + hrow] = l_part;
+    }
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      ow[(warp * kMaxR + hrow) * D + 8 * n + 2 * c4] = oacc[n][0];
+      ow[(warp * kMaxR + hrow) * D + 8 * n + 2 * c4 + 1] = oacc[n][1];
+    }
+  }
+  named_sync_consumers();
+  const size_t pbase = (((size_t)b * args.Hkv + g) * args.splits + split) * r;
+  for (int idx = threadIdx.x; idx < r * D; idx += 128) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, mw[w * kMaxR + h]);
+    float o = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float mwv = mw[w * kMaxR + h];
+      const float wt = (mwv == -INFINITY) ? 0.f : ex2_approx(mwv - M);
+      o += wt * ow[(w * kMaxR + h) * D + d];
+      l += wt * lw[w * kMaxR + h];
+    }
+    args.part_o[(pbase + h) * D + d] = o;
+    if (d == 0) args.part_ml[pbase + h] = make_float2(M, l);
+  }
+
+  // ---------------------------------------------------------- last CTA merges
+  __threadfence();
+  named_sync_consumers();
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(&args.counters[b * args.Hkv + g], 1);
+    *ticket_slot = (prev == args.splits - 1) ? 1 : 0;
+  }
+  named_sync_consumers();
+  if (*ticket_slot == 0) return;
+  __threadfence();
+  const size_t sbase_p = ((size_t)b * args.Hkv + g) * args.splits;
+  for (int h = warp; h < r; h += 4) {
+    float M = -INFINITY;
+    for (int sp = lane; sp < args.splits; sp += 32) M = fmaxf(M, __ldcg(&args.part_ml[(sbase_p + sp) * r + h]).x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float l = 0.f;
+    for (int sp = lane; sp < args.splits; sp += 32) {
+      const float2 ml = __ldcg(&args.part_ml[(sbase_p + sp) * r + h]);
+      l += (ml.x == -INFINITY) ? 0.f : ml.y * ex2_approx(ml.x - M);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    for (int d = lane; d < D; d += 32) {
+      float acc = 0.f;
+      for (int sp = 0; sp < args.splits; ++sp) {
+        const float mx = __ldcg(&args.part_ml[(sbase_p + sp) * r + h]).x;
+        const float wt = (mx == -INFINITY) ? 0.f : ex2_approx(mx - M);
+        acc += wt * __ldcg(&args.part_o[((sbase_p + sp) * r + h) * D + d]);
+      }
+      args.o[((size_t)b * args.Hq + g * r + h) * D + d] = __float2bfloat16_rn(acc * inv);
+    }
+    if (lane == 0 && args.lse != nullptr)
+      args.lse[(size_t)b * args.Hq + g * r + h] = (M + __log2f(l)) * 0.69314718055994531f;
+  }
+  if (threadIdx.x == 0) args.counters[b * args.Hkv + g] = 0;  // ready for the next call
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeArgs& a, int D,
+                          cudaStream_t stream) {
+  dim3 grid(a.splits, a.Hkv, a.B);
+  if (D == 128) {
+    auto k = bifocal_decode_kernel<128>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<128>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kDecThreads, DecCfg<128>::kSmem, stream>>>(tm_k, tm_v, a);
+  } else {
+    auto k = bifocal_decode_kernel<64>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<64>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kDecThreads, DecCfg<64>::kSmem, stream>>>(tm_k, tm_v, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace jl

@@ -1,0 +1,331 @@
+// C ABI of libjetlong.so: argument checks, position maps, scratch layout,
+// tensor-map encoding and kernel launches.  See include/jl_api.h.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/jl_api.h"
+#include "jl_kernels.cuh"
+
+namespace {
+
+using jl::DecodeArgs;
+using jl::PrefillArgs;
+using jl::RotateArgs;
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D 16-bit map over [B, rows, H, D] (innermost first: D, H, rows, B) with a
+// {64, 1, box_rows, 1} box and 128-byte swizzle.
+bool encode_16bit_4d(CUtensorMap* map, const void* base, int D, int H, int64_t rows, int B, int box_rows,
+                     CUtensorMapDataType dtype) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)rows * H * D * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_bf16_4d(CUtensorMap* map, const void* base, int D, int H, int64_t rows, int B, int box_rows) {
+  return encode_16bit_4d(map, base, D, H, rows, B, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+bool encode_f16_4d(CUtensorMap* map, const void* base, int D, int H, int64_t rows, int B, int box_rows) {
+  return encode_16bit_4d(map, base, D, H, rows, B, box_rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+void fill_theta(double* theta, int D, double base) {
+  for (int t = 0; t < D / 2; ++t) theta[t] = std::pow(base, -2.0 * t / D);
+}
+
+int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained, double rope_base, int mode) {
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || w0 < 0 || w_pretrained < 1) return JL_ERR_INVALID_ARG;
+  if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return JL_ERR_INVALID_ARG;
+  if (mode != JL_QSHIFT_NONE && mode != JL_QSHIFT_SELF_EXTEND) return JL_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
+  if (L > (1 << 30)) return JL_ERR_UNSUPPORTED;
+  return JL_OK;
+}
+
+float resolve_scale(float s, int D) { return s == 0.f ? 1.0f / std::sqrt((float)D) : s; }
+
+// Decode split count: about two CTAs per SM over all (batch, KV head) pairs.
+int decode_splits_max(int B, int Hkv) {
+  const int target = 2 * device_sms();
+  int s = (target + B * Hkv - 1) / (B * Hkv);
+  if (s < 1) s = 1;
+  if (s > 4096) s = 4096;
+  return s;
+}
+
+struct DecodeLayout {
+  size_t counters, ml, o, total;
+};
+DecodeLayout decode_layout(int B, int Hq, int Hkv, int D, int splits) {
+  const int r = Hq / Hkv;
+  DecodeLayout lay;
+  lay.counters = 0;
+  lay.ml = round_up((size_t)B * Hkv * sizeof(int));
+  lay.o = lay.ml + round_up((size_t)B * Hkv * splits * r * sizeof(float2));
+  lay.total = lay.o + round_up((size_t)B * Hkv * splits * r * D * sizeof(float));
+  return lay;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* jl_status_string(int status) {
+  switch (status) {
+    case JL_OK: return "ok";
+    case JL_ERR_INVALID_ARG: return "invalid argument";
+    case JL_ERR_UNSUPPORTED: return "unsupported shape";
+    case JL_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case JL_ERR_WORKSPACE: return "workspace missing or too small";
+    case JL_ERR_CUDA: return "CUDA error";
+    case JL_ERR_DEVICE_TIMEOUT: return "device pipeline timeout";
+    default: return "unknown status";
+  }
+}
+
+int jl_group_size(int64_t L, int64_t w_pretrained, int64_t* G_out) {
+  if (G_out == nullptr || L < 0 || w_pretrained < 1) return JL_ERR_INVALID_ARG;
+  *G_out = jl::group_size(L, w_pretrained);
+  return JL_OK;
+}
+
+int jl_remote_positions(int64_t L, int64_t w0, int64_t w_pretrained, int mode, int32_t* q_pos_out,
+                        int32_t* k_pos_out) {
+  if (L < 1 || w0 < 0 || w_pretrained < 1) return JL_ERR_INVALID_ARG;
+  if (mode != JL_QSHIFT_NONE && mode != JL_QSHIFT_SELF_EXTEND) return JL_ERR_INVALID_ARG;
+  const int64_t G = jl::group_size(L, w_pretrained);
+  const int64_t shift = jl::query_shift(w0, G, mode);
+  if ((L - 1) / G + shift > INT32_MAX) return JL_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < L; ++i) {
+    if (q_pos_out) q_pos_out[i] = (int32_t)jl::query_remote(i, G, shift);
+    if (k_pos_out) k_pos_out[i] = (int32_t)jl::key_remote(i, G);
+  }
+  return JL_OK;
+}
+
+size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
+  return round_up((size_t)B * L * Hq * head_dim * 2) + round_up((size_t)B * L * Hkv * head_dim * 2);
+}
+
+namespace {
+
+// Shared argument checks of the prefill entry points.
+int prefill_checks(const void* q, const void* k, const void* v, int B, int L, int Hq, int Hkv, int D, int w0,
+                   int w_pretrained, double rope_base, int mode) {
+  int st = common_checks(B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+  if (st != JL_OK) return st;
+  if (!q || !k || !v) return JL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return JL_ERR_ALIGNMENT;
+  return JL_OK;
+}
+
+__half* q_rem_ptr(void* ws) { return reinterpret_cast<__half*>(ws); }
+__half* k_rem_ptr(void* ws, int B, int L, int Hq, int D) {
+  return reinterpret_cast<__half*>(reinterpret_cast<char*>(ws) + round_up((size_t)B * L * Hq * D * 2));
+}
+
+}  // namespace
+
+int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, int Hkv, int head_dim, int w0,
+                          int w_pretrained, double rope_base, int mode, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  const int D = head_dim;
+  int st = prefill_checks(q, k, k, B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+  if (st != JL_OK) return st;
+  const int64_t G = jl::group_size(L, w_pretrained);
+  if (jl::all_local(L, w0, G)) return JL_OK;  // nothing to correct
+  if (!workspace || workspace_bytes < jl_prefill_workspace_bytes(B, L, Hq, Hkv, D)) return JL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  RotateArgs ra;
+  std::memset(&ra, 0, sizeof(ra));
+  fill_theta(ra.theta, D, rope_base);
+  ra.G = G;
+  ra.shift = jl::query_shift(w0, G, mode);
+  ra.B = B;
+  ra.L = L;
+  // queries that have a remote key: i >= w0
+  ra.x = reinterpret_cast<const __nv_bfloat16*>(q);
+  ra.y = q_rem_ptr(workspace);
+  ra.H = Hq;
+  ra.row_begin = w0;
+  ra.row_end = L;
+  ra.is_query = 1;
+  if (jl::launch_rotate_rows(ra, D, s) != cudaSuccess) return JL_ERR_CUDA;
+  // keys that have a remote query: j <= L - 1 - w0
+  ra.x = reinterpret_cast<const __nv_bfloat16*>(k);
+  ra.y = k_rem_ptr(workspace, B, L, Hq, D);
+  ra.H = Hkv;
+  ra.row_begin = 0;
+  ra.row_end = L - w0;
+  ra.is_query = 0;
+  if (jl::launch_rotate_rows(ra, D, s) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
+                         int Hkv, int head_dim, int w0, int w_pretrained, float softmax_scale, int mode,
+                         const void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
+  const int D = head_dim;
+  int st = prefill_checks(q, k, v, B, L, Hq, Hkv, D, w0, w_pretrained, 10000.0, mode);
+  if (st != JL_OK) return st;
+  if (!o) return JL_ERR_INVALID_ARG;
+  if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
+  const int64_t G = jl::group_size(L, w_pretrained);
+  const bool all_local = jl::all_local(L, w0, G);
+  if (!all_local) {
+    if (!workspace || workspace_bytes < jl_prefill_workspace_bytes(B, L, Hq, Hkv, D)) return JL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
+  }
+  CUtensorMap tq, tqr, tk, tkr, tv;
+  if (!encode_bf16_4d(&tq, q, D, Hq, L, B, 128) || !encode_bf16_4d(&tk, k, D, Hkv, L, B, 128) ||
+      !encode_bf16_4d(&tv, v, D, Hkv, L, B, 128))
+    return JL_ERR_CUDA;
+  if (!all_local) {
+    void* ws = const_cast<void*>(workspace);
+    if (!encode_f16_4d(&tqr, q_rem_ptr(ws), D, Hq, L, B, 128) ||
+        !encode_f16_4d(&tkr, k_rem_ptr(ws, B, L, Hq, D), D, Hkv, L, B, 128))
+      return JL_ERR_CUDA;
+  } else {
+    tqr = tq;
+    tkr = tk;
+  }
+  const int r = Hq / Hkv;
+  PrefillArgs pa;
+  std::memset(&pa, 0, sizeof(pa));
+  pa.o = reinterpret_cast<__nv_bfloat16*>(o);
+  pa.lse = lse;
+  pa.dev_error = dev_error;
+  pa.B = B;
+  pa.L = L;
+  pa.Hq = Hq;
+  pa.Hkv = Hkv;
+  pa.r = r;
+  pa.nh = (r % 2 == 0) ? 2 : 1;
+  pa.num_mb = (L + 127) / 128;
+  pa.all_local = all_local ? 1 : 0;
+  pa.w0 = all_local ? (1 << 30) : w0;
+  pa.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
+  if (jl::launch_prefill(tq, tqr, tk, tkr, tv, pa, D, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int jl_bifocal_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
+                       int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,
+                       int mode, void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
+  // Validate everything before the first launch.
+  const int D = head_dim;
+  int st = prefill_checks(q, k, v, B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+  if (st != JL_OK) return st;
+  if (!o) return JL_ERR_INVALID_ARG;
+  if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
+  const int64_t G = jl::group_size(L, w_pretrained);
+  if (!jl::all_local(L, w0, G)) {
+    if (!workspace || workspace_bytes < jl_prefill_workspace_bytes(B, L, Hq, Hkv, D)) return JL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
+  }
+  st = jl_prefill_correction(q, k, B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode, workspace,
+                             workspace_bytes, stream);
+  if (st != JL_OK) return st;
+  return jl_prefill_attention(q, k, v, o, lse, B, L, Hq, Hkv, D, w0, w_pretrained, softmax_scale, mode, workspace,
+                              workspace_bytes, dev_error, stream);
+}
+
+size_t jl_decode_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || head_dim < 1 || Hq % Hkv) return 0;
+  return decode_layout(B, Hq, Hkv, head_dim, decode_splits_max(B, Hkv)).total;
+}
+
+int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                      float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
+                      double rope_base, float softmax_scale, int mode, void* workspace, size_t workspace_bytes,
+                      int* dev_error, void* stream) {
+  const int D = head_dim;
+  int st = common_checks(B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+  if (st != JL_OK) return st;
+  if (!q || !k_cache || !v_cache || !o) return JL_ERR_INVALID_ARG;
+  if (cache_len < L || cache_len > (int64_t)1 << 31) return JL_ERR_INVALID_ARG;
+  if (Hq / Hkv > 8) return JL_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (lse && ((uintptr_t)lse & 3u)))
+    return JL_ERR_ALIGNMENT;
+  const int ntiles = (L + 63) / 64;
+  int splits = decode_splits_max(B, Hkv);
+  if (splits > ntiles) splits = ntiles;
+  const DecodeLayout lay = decode_layout(B, Hq, Hkv, D, decode_splits_max(B, Hkv));
+  if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
+
+  const int64_t G = jl::group_size(L, w_pretrained);
+  const bool all_local = jl::all_local(L, w0, G);
+  const int64_t shift = jl::query_shift(w0, G, mode);
+
+  CUtensorMap tk, tv;
+  if (!encode_bf16_4d(&tk, k_cache, D, Hkv, cache_len, B, 64) ||
+      !encode_bf16_4d(&tv, v_cache, D, Hkv, cache_len, B, 64))
+    return JL_ERR_CUDA;
+
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  char* ws = reinterpret_cast<char*>(workspace);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.counters = reinterpret_cast<int*>(ws + lay.counters);
+  a.part_ml = reinterpret_cast<float2*>(ws + lay.ml);
+  a.part_o = reinterpret_cast<float*>(ws + lay.o);
+  a.dev_error = dev_error;
+  a.B = B;
+  a.L = L;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.r = Hq / Hkv;
+  a.splits = splits;
+  a.ntiles = ntiles;
+  a.w0 = all_local ? (1 << 30) : w0;
+  a.all_local = all_local ? 1 : 0;
+  a.G = G;
+  a.dq = jl::query_remote(L - 1, G, shift) - (L - 1);
+  a.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
+  fill_theta(a.theta, D, rope_base);
+  if (jl::launch_decode(tk, tv, a, D, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,437 @@
+// Fused Dynamic Bifocal RoPE prefill for sm_100a.
+//
+// Causal GQA attention where a (query i, key j) pair with i - j < w0 is scored
+// with the base-rotated Q and K (exact base RoPE), and every other causal pair
+// with the remote-rotated rows R(p_q(i)) q and R(f(j)) k (Jet-Long review,
+// "Method"; gist.science summary, "Methodologie §1").  The remote rows come
+// from the correction pass in rope_rotate.cu, in fp16; local products are
+// bf16 x bf16, remote ones fp16 x fp16, P V is bf16 x bf16, all fp32-accumulated.
+//
+// Instead of the pages' three FlashAttention calls merged by inclusion-exclusion,
+// each 128x128 (query block, key block) tile is classified by its range of
+// i - j: wholly local, wholly remote, or straddling the band edge.  A tile is
+// visited once per score set it needs ("pass"): local passes read Q / K, remote
+// passes read Q_rem / K_rem, and a straddling tile gets one pass of each with
+// complementary masks.  Both passes feed the same online softmax, so no score
+// is counted twice and nothing is subtracted.
+//
+// CTA = one 128-row query block of NH (1 or 2) query heads that share a KV head.
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q (base, later remote) and a 2-stage K / V ring
+//   warp 1      tcgen05 MMA issuer; owns the TMEM allocation
+//   warps 4-7   softmax for head 0 (thread = query row = TMEM lane)
+//   warps 8-11  softmax for head 1
+// TMEM columns: S_h at 128 h, O_h at 128 NH + D h.  P (bf16) overwrites the
+// first 64 columns of S_h and is the A operand of O_h += P V from TMEM.
+// Per pass the MMA order is S0(i), PV1(i-1), S1(i), PV0(i): each softmax group
+// works on its S while the tensor core runs the other head's two products.
+#include "jl_kernels.cuh"
+
+namespace jl {
+
+namespace {
+
+constexpr int kBM = 128;  // query rows per block
+constexpr int kBN = 128;  // keys per tile
+constexpr int kStages = 2;
+constexpr int kThreads = 384;
+constexpr int kChunkBytes = 128 * 128;  // one 128-row x 128-byte swizzled slab
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;  // 64-element (128 B) slabs per row
+  static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr int kUsed = kBarOff + 256;
+  // Ask for enough shared memory that only one CTA fits per SM: each CTA
+  // allocates up to 512 TMEM columns.
+  static constexpr int kSmem = (kUsed < 120 * 1024 ? 120 * 1024 : kUsed) + 1024;
+};
+
+// barrier slots
+enum {
+  kQFull = 0,
+  kQEmpty = 1,
+  kKFull = 2,
+  kKEmpty = kKFull + kStages,
+  kVFull = kKEmpty + kStages,
+  kVEmpty = kVFull + kStages,
+  kSFull = kVEmpty + kStages,  // 2
+  kPFull = kSFull + 2,         // 2
+  kOFinal = kPFull + 2,
+  kDrain = kOFinal + 1,
+  kNumBars = kDrain + 1
+};
+static_assert(kNumBars * 8 <= 192, "barrier block overflow");
+
+// Pass schedule of one query block mb: n_loc local passes on key blocks
+// mb, mb-1, ... then n_rem remote passes on key blocks mb - a_min, ..., 0.
+struct Sched {
+  int n_loc, n_rem, a_min;
+};
+
+__device__ __forceinline__ Sched make_sched(int mb, int w0, bool all_local) {
+  Sched s;
+  if (all_local) {
+    s.n_loc = mb + 1;
+    s.n_rem = 0;
+    s.a_min = mb + 1;
+    return s;
+  }
+  // block distance a = mb - nb spans i - j in [128a - 127, 128a + 127]
+  // local pairs exist iff w0 > 0 and 128a - 127 < w0
+  s.n_loc = (w0 > 0) ? min(mb, (w0 + 126) / 128) + 1 : 0;
+  // remote pairs exist iff 128a + 127 >= w0
+  s.a_min = w0 / 128;
+  s.n_rem = max(0, mb - s.a_min + 1);
+  return s;
+}
+
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
+  // Used only after an abort: wait (up to ~100 ms) for async work already in
+  // flight so the CTA never exits while a copy or an MMA still targets it.
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > 100000000ull) return false;
+  }
+  return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
+                           const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
+                           const __grid_constant__ CUtensorMap tm_v, const PrefillArgs args) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 196);
+  auto bar = [&](int i) -> uint32_t { return smem_addr(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int NH = args.nh;
+  const int hq0 = blockIdx.x * NH;
+  const int mb = args.num_mb - 1 - (int)blockIdx.y;  // heaviest blocks first
+  const int b = blockIdx.z;
+  const int kvh = hq0 / args.r;
+  const uint32_t ncols = NH == 2 ? 512u : 256u;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(kQFull), 1);
+    mbar_init(bar(kQEmpty), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kKFull + s), 1);
+      mbar_init(bar(kKEmpty + s), 1);
+      mbar_init(bar(kVFull + s), 1);
+      mbar_init(bar(kVEmpty + s), 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(kSFull + h), 1);
+      mbar_init(bar(kPFull + h), 128);
+    }
+    mbar_init(bar(kOFinal), 1);
+    mbar_init(bar(kDrain), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const Sched sc = make_sched(mb, args.w0, args.all_local != 0);
+  const int npass = sc.n_loc + sc.n_rem;
+  const bool q_switch = sc.n_loc > 0 && sc.n_rem > 0;
+  const int w0 = args.w0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_qr);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_kr);
+      tma_prefetch_map(&tm_v);
+      const uint32_t q_bytes = (uint32_t)(NH * C::kTileBytes);
+      auto load_q = [&](const CUtensorMap* m) {
+        mbar_arrive_expect_tx(bar(kQFull), q_bytes);
+        for (int hh = 0; hh < NH; ++hh)
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sbase + C::kQOff + hh * C::kTileBytes + c * kChunkBytes, m, bar(kQFull), c * 64,
+                        hq0 + hh, mb * kBM, b);
+      };
+      load_q(sc.n_loc > 0 ? &tm_q : &tm_qr);
+      int q_loads = 1;
+      int k_last = -1, v_last = -1;  // last passes whose K / V copies were issued
+      bool ok = true;
+      for (int p = 0; p < npass; ++p) {
+        const int s = p % kStages;
+        const uint32_t ph = (uint32_t)(p / kStages) & 1u;
+        const bool remote = p >= sc.n_loc;
+        const int a = remote ? sc.a_min + (p - sc.n_loc) : p;
+        const int nb = mb - a;
+        if (q_switch && p == sc.n_loc) {
+          if (!(ok = mbar_wait(bar(kQEmpty), 0, abort_flag, args.dev_error))) break;
+          load_q(&tm_qr);
+          ++q_loads;
+        }
+        if (!(ok = mbar_wait(bar(kKEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
+        mbar_arrive_expect_tx(bar(kKFull + s), (uint32_t)C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sbase + C::kKOff + s * C::kTileBytes + c * kChunkBytes, remote ? &tm_kr : &tm_k,
+                      bar(kKFull + s), c * 64, kvh, nb * kBN, b);
+        k_last = p;
+        if (!(ok = mbar_wait(bar(kVEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
+        mbar_arrive_expect_tx(bar(kVFull + s), (uint32_t)C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sbase + C::kVOff + s * C::kTileBytes + c * kChunkBytes, &tm_v, bar(kVFull + s), c * 64,
+                      kvh, nb * kBN, b);
+        v_last = p;
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA can exit.
+        drain_wait(bar(kQFull), (uint32_t)(q_loads - 1) & 1u);
+        for (int p = max(0, k_last - kStages + 1); p <= k_last; ++p)
+          drain_wait(bar(kKFull + p % kStages), (uint32_t)(p / kStages) & 1u);
+        for (int p = max(0, v_last - kStages + 1); p <= v_last; ++p)
+          drain_wait(bar(kVFull + p % kStages), (uint32_t)(p / kStages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s_loc = make_idesc_16bit(kBM, kBN, false, false);  // bf16 Q K
+      const uint32_t id_s_rem = make_idesc_16bit(kBM, kBN, false, true);   // fp16 Q_rem K_rem
+      const uint32_t id_pv = make_idesc_16bit(kBM, D, true, false);        // bf16 P V
+      bool ok = mbar_wait(bar(kQFull), 0, abort_flag, args.dev_error);
+      auto s_col = [&](int h) -> uint32_t { return (uint32_t)(h * 128); };
+      auto o_col = [&](int h) -> uint32_t { return (uint32_t)(NH * 128 + h * D); };
+
+      auto issue_s = [&](int h, int p) -> bool {
+        const int s = p % kStages;
+        const uint32_t ph = (uint32_t)(p / kStages) & 1u;
+        if (h == 0) {
+          if (q_switch && p == sc.n_loc && !mbar_wait(bar(kQFull), 1, abort_flag, args.dev_error)) return false;
+          if (!mbar_wait(bar(kKFull + s), ph, abort_flag, args.dev_error)) return false;
+          tc_fence_after();
+        }
+        const uint32_t qa = sbase + C::kQOff + h * C::kTileBytes;
+        const uint32_t ka = sbase + C::kKOff + s * C::kTileBytes;
+        const uint32_t id_s = p >= sc.n_loc ? id_s_rem : id_s_loc;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
+          mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+                 id_s, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kSFull + h));
+        if (h == NH - 1) {
+          tc_commit(bar(kKEmpty + s));
+          if (q_switch && p == sc.n_loc - 1) tc_commit(bar(kQEmpty));
+        }
+        return true;
+      };
+      auto issue_pv = [&](int h, int p) -> bool {
+        const int s = p % kStages;
+        const uint32_t ph = (uint32_t)(p / kStages) & 1u;
+        if (h == 0 && !mbar_wait(bar(kVFull + s), ph, abort_flag, args.dev_error)) return false;
+        if (!mbar_wait(bar(kPFull + h), (uint32_t)p & 1u, abort_flag, args.dev_error)) return false;
+        tc_fence_after();
+        const uint32_t va = sbase + C::kVOff + s * C::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks) {
+          // V tile is MN-major for this product: 64-dim slabs kChunkBytes apart
+          // (leading offset), 8-key groups 1024 B apart (stride offset).
+          mma_ts(tmem + o_col(h), tmem + s_col(h) + (uint32_t)(ks * 8),
+                 make_sdesc_sw128(va + (uint32_t)(ks * 2048), kChunkBytes, 1024), id_pv,
+                 (p > 0 || ks > 0) ? 1u : 0u);
+        }
+        if (h == NH - 1) tc_commit(bar(kVEmpty + s));
+        return true;
+      };
+
+      if (ok) {
+        if (NH == 2) {
+          ok = issue_s(0, 0) && issue_s(1, 0) && issue_pv(0, 0);
+          for (int p = 1; p < npass && ok; ++p) {
+            ok = issue_s(0, p) && issue_pv(1, p - 1) && issue_s(1, p) && issue_pv(0, p);
+          }
+          if (ok) ok = issue_pv(1, npass - 1);
+        } else {
+          for (int p = 0; p < npass && ok; ++p) ok = issue_s(0, p) && issue_pv(0, p);
+        }
+      }
+      // Every product issued must have completed before TMEM is released.
+      if (ok) {
+        tc_commit(bar(kOFinal));
+        drain_wait(bar(kOFinal), 0);
+      } else {
+        tc_commit(bar(kDrain));
+        drain_wait(bar(kDrain), 0);
+      }
+    }
+  } else if (warp >= 4 && ((warp - 4) >> 2) < NH) {
+    // ------------------------------------------------------------ softmax
+    const int h = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int hq = hq0 + h;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + (uint32_t)(h * 128);
+    const uint32_t o_addr = tmem + lane_off + (uint32_t)(NH * 128 + h * D);
+    const float sl2 = args.scale_log2;
+    float m_used = -INFINITY;
+    float l_sum = 0.f;
+    bool ok = true;
+
+    for (int p = 0; p < npass; ++p) {
+      ok = mbar_wait(bar(kSFull + h), (uint32_t)p & 1u, abort_flag, args.dev_error);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const bool remote = p >= sc.n_loc;
+      const int a = remote ? sc.a_min + (p - sc.n_loc) : p;
+
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]) * sl2;
+
+      const bool need_mask = remote ? (128 * a - 127 < w0) : (a == 0 || 128 * a + 127 >= w0);
+      if (need_mask) {
+        const int dd = 128 * a + row;  // i - j = dd - col
+#pragma unroll
+        for (int col = 0; col < 128; ++col) {
+          const int rel = dd - col;
+          const bool keep = remote ? (rel >= w0) : (rel >= 0 && rel < w0);
+          if (!keep) x[col] = -INFINITY;
+        }
+      }
+      float mt = x[0];
+#pragma unroll
+      for (int col = 1; col < 128; ++col) mt = fmaxf(mt, x[col]);
+      const float m_new = fmaxf(m_used, mt);
+      float alpha = 1.f;
+      bool rescale_o = false;
+      // Lazy rescaling: keep the exponent offset until the row max has grown
+      // by more than 2^8; p <= 256 stays exact enough in fp32 / bf16.
+      if (m_new > m_used + 8.f) {
+        if (m_used != -INFINITY) {
+          alpha = ex2_approx(m_used - m_new);
+          rescale_o = true;
+        } else {
+          alpha = 0.f;
+        }
+        l_sum *= alpha;
+        m_used = m_new;
+      }
+      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+
+      float rs = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float p0 = ex2_approx(x[half * 64 + 2 * k] - msub);
+          const float p1 = ex2_approx(x[half * 64 + 2 * k + 1] - msub);
+          rs += p0 + p1;
+          pk[k] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_addr + half * 32, pk);
+      }
+      l_sum += rs;
+
+      if (__any_sync(0xffffffffu, rescale_o) && p > 0) {
+        // O_h(p-1) is final here: its product was issued before S_h(p).
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + c * 32, ov);
+          tmem_ld_wait(ov);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+          tmem_st32(o_addr + c * 32, ov);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kPFull + h));
+    }
+
+    if (ok) {
+      ok = mbar_wait(bar(kOFinal), 0, abort_flag, args.dev_error);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int i = mb * kBM + row;
+      const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      __nv_bfloat16* orow = args.o + (((size_t)b * args.L + i) * args.Hq + hq) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(o_addr + c * 32, ov);
+        tmem_ld_wait(ov);
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          w[k] = pack_bf16x2(__uint_as_float(ov[2 * k]) * inv, __uint_as_float(ov[2 * k + 1]) * inv);
+        if (i < args.L) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        }
+      }
+      if (args.lse != nullptr && i < args.L) {
+        const float m = (m_used == -INFINITY) ? 0.f : m_used;
+        args.lse[((size_t)b * args.Hq + hq) * args.L + i] = (m + __log2f(l_sum)) * 0.69314718055994531f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
+                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const PrefillArgs& a,
+                           int D, cudaStream_t stream) {
+  dim3 grid(a.Hq / a.nh, a.num_mb, a.B);
+  if (D == 128) {
+    auto k = bifocal_prefill_kernel<128>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<128>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, Cfg<128>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, a);
+  } else {
+    auto k = bifocal_prefill_kernel<64>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<64>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, Cfg<64>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace jl

@@ -1,0 +1,91 @@
+"""Shared helpers for the GPU parity tests: run the library through the C-ABI
+binding and compare with the fp64 oracle on the same seeded inputs."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import jetlong_oracle as jo
+from rope_context_extension_b200 import jetlong as jl
+from rope_context_extension_b200 import synthetic
+
+# Tolerances against the fp64 oracle (bf16 outputs, fp32 LSE).
+O_MAX_ABS = 2e-2
+O_MEAN_ABS = 2e-3
+LSE_MAX_ABS = 1e-3
+
+MODES = {jo.MODE_NONE: jl.JL_QSHIFT_NONE, jo.MODE_SELF_EXTEND: jl.JL_QSHIFT_SELF_EXTEND}
+
+
+def run_prefill(q, k, v, *, w0, W, base, mode=jo.MODE_SELF_EXTEND, scale=0.0):
+    """Run jl_bifocal_prefill on CPU bf16 inputs; returns (O float32 CPU, LSE CPU, dev_error)."""
+    dev = torch.device("cuda")
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    ws = torch.empty(jl.jl_prefill_workspace_bytes(B, L, Hq, Hkv, D), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    jl.jl_bifocal_prefill(qd, kd, vd, o, lse, w0=w0, w_pretrained=W, rope_base=base, softmax_scale=scale,
+                          mode=MODES[mode], workspace=ws, dev_error=err)
+    torch.cuda.synchronize()
+    return o.float().cpu(), lse.cpu(), int(err.item())
+
+
+def run_decode(q, kc, vc, *, L, w0, W, base, mode=jo.MODE_SELF_EXTEND, scale=0.0, workspace=None):
+    dev = torch.device("cuda")
+    B, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    qd, kd, vd = q.to(dev), kc.to(dev), vc.to(dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.zeros(jl.jl_decode_workspace_bytes(B, L, Hq, Hkv, D), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    jl.jl_bifocal_decode(qd, kd, vd, o, lse, L=L, w0=w0, w_pretrained=W, rope_base=base, softmax_scale=scale,
+                         mode=MODES[mode], workspace=workspace, dev_error=err)
+    torch.cuda.synchronize()
+    return o.float().cpu(), lse.cpu(), int(err.item())
+
+
+def assert_close(o_gpu, o_ref, lse_gpu, lse_ref, what=""):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    err = np.abs(o_gpu - o_ref)
+    lerr = np.abs(np.asarray(lse_gpu, dtype=np.float64) - np.asarray(lse_ref, dtype=np.float64))
+    msg = f"{what}: O max {err.max():.3e} mean {err.mean():.3e}; LSE max {lerr.max():.3e}"
+    assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(lse_gpu)), msg
+    assert err.max() <= O_MAX_ABS, msg
+    assert err.mean() <= O_MEAN_ABS, msg
+    assert lerr.max() <= LSE_MAX_ABS, msg
+    return err.max(), err.mean(), lerr.max()
+
+
+def sample_rows(L: int, w0: int, n: int, seed: int = 0):
+    """Seeded query rows plus the band and tile edges."""
+    rng = np.random.default_rng(seed)
+    edges = {0, L - 1, w0 - 1, w0, w0 + 1, 127, 128, L // 2}
+    for m in (1, 2, 7, L // 128 - 1, L // 128):
+        edges |= {128 * m - 1, 128 * m}
+    rows = set(int(x) for x in edges if 0 <= x < L)
+    rows |= set(int(x) for x in rng.choice(L, size=min(n, L), replace=False))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def oracle_prefill_rows(q, k, v, rows, heads, p: jo.BifocalParams):
+    """Oracle rows for the listed heads (b = 0): dict h -> (O[n, d], LSE[n])."""
+    Hq, Hkv = q.shape[2], k.shape[2]
+    r = Hq // Hkv
+    out = {}
+    by_g = {}
+    for h in heads:
+        by_g.setdefault(h // r, []).append(h)
+    for g, hs in by_g.items():
+        kg = k[0, :, g, :].double().numpy()
+        vg = v[0, :, g, :].double().numpy()
+        for h in hs:
+            qh = q[0, rows, h, :].double().numpy()
+            out[h] = jo.attention_rows(qh, rows, kg, vg, p)
+    return out

@@ -1,0 +1,201 @@
+"""GPU parity: the CUDA path through the C-ABI against the fp64 oracle.
+
+Tolerances (bf16 outputs vs fp64): O max-abs 2e-2 and mean-abs 2e-3, LSE
+max-abs 1e-3.  Small cases compare every output; the full-size workloads
+compare seeded samples of query rows (rows are independent, so each sampled
+row is an exact oracle row), always including band and tile edges.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import jetlong_oracle as jo
+from rope_context_extension_b200 import synthetic
+from tests.gpu_helpers import (assert_close, oracle_prefill_rows, run_decode, run_prefill, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from rope_context_extension_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+# ---------------------------------------------------------------------------
+# prefill, every output compared
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [jo.MODE_SELF_EXTEND, jo.MODE_NONE])
+def test_prefill_tiny_workload(mode):
+    # batch 1, 2 q heads / 1 kv head, d 64, L 512, w_pretrained 128 (G 4), w0 32, base 1e4, seed 0
+    q, k, v = synthetic.prefill_inputs(1, 512, 2, 1, 64, seed=0)
+    p = jo.BifocalParams(L=512, w0=32, w_pretrained=128, base=10000.0, mode=mode)
+    o, lse, err = run_prefill(q, k, v, w0=32, W=128, base=10000.0, mode=mode)
+    assert err == 0
+    o_ref, lse_ref = jo.prefill_dense(q.float().numpy(), k.float().numpy(), v.float().numpy(), p)
+    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, "tiny")
+
+
+CASES = [
+    # B, L, Hq, Hkv, D, W, w0, mode, outliers
+    (1, 1000, 4, 2, 128, 300, 200, jo.MODE_SELF_EXTEND, 0.0),   # ragged, several tiles, G 4
+    (1, 1000, 4, 2, 128, 300, 200, jo.MODE_NONE, 0.0),
+    (2, 777, 3, 1, 64, 200, 77, jo.MODE_SELF_EXTEND, 0.01),     # odd GQA ratio (one head per CTA), B 2
+    (1, 640, 2, 2, 128, 100, 0, jo.MODE_SELF_EXTEND, 0.01),     # w0 = 0: every pair remote, MHA
+    (1, 600, 8, 2, 128, 90, 600, jo.MODE_SELF_EXTEND, 0.0),     # w0 = L: plain causal RoPE
+    (1, 900, 4, 1, 128, 1024, 64, jo.MODE_SELF_EXTEND, 0.01),   # G = 1: plain causal RoPE
+    (1, 129, 2, 1, 64, 50, 128, jo.MODE_SELF_EXTEND, 0.0),      # one row past a tile
+    (1, 1, 2, 1, 128, 16, 0, jo.MODE_SELF_EXTEND, 0.0),         # single token
+    (1, 1300, 8, 2, 128, 260, 1, jo.MODE_SELF_EXTEND, 0.01),    # w0 = 1: only the diagonal is local
+]
+
+
+@pytest.mark.parametrize("B,L,Hq,Hkv,D,W,w0,mode,outl", CASES)
+def test_prefill_small_cases(B, L, Hq, Hkv, D, W, w0, mode, outl):
+    q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=L + w0, outlier_frac=outl)
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=10000.0, mode=mode)
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=10000.0, mode=mode)
+    assert err == 0
+    o_ref, lse_ref = jo.prefill_dense(q.float().numpy(), k.float().numpy(), v.float().numpy(), p)
+    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"L{L} w0{w0}")
+
+
+def test_prefill_plain_mode_is_identical_across_equivalent_calls():
+    # G = 1 and w0 >= L both select plain causal RoPE: same kernels, same bits.
+    q, k, v = synthetic.prefill_inputs(1, 700, 4, 2, 128, seed=3)
+    o1, l1, _ = run_prefill(q, k, v, w0=10, W=700, base=1e6)
+    o2, l2, _ = run_prefill(q, k, v, w0=700, W=100, base=1e6)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_prefill_deterministic():
+    q, k, v = synthetic.prefill_inputs(1, 1024, 4, 1, 128, seed=4)
+    a = run_prefill(q, k, v, w0=100, W=256, base=1e6)
+    b = run_prefill(q, k, v, w0=100, W=256, base=1e6)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------------------
+# prefill at the full workload sizes, sampled rows
+# ---------------------------------------------------------------------------
+
+FULL = [
+    # name, B, L, Hq, Hkv, W, w0
+    ("qwen3-1.7b-64k", 1, 65536, 16, 8, 32768, 4096),
+    ("qwen3-8b-128k", 1, 131072, 32, 8, 32768, 4096),
+]
+
+
+@pytest.mark.parametrize("name,B,L,Hq,Hkv,W,w0", FULL)
+def test_prefill_full_size_sampled(name, B, L, Hq, Hkv, W, w0):
+    q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, 128, seed=0)
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6)
+    assert err == 0
+    rows = sample_rows(L, w0, 40, seed=1)
+    heads = sorted({0, 1, Hq // 2 + 1, Hq - 1})
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+    ref = oracle_prefill_rows(q, k, v, rows, heads, p)
+    for h in heads:
+        o_ref, lse_ref = ref[h]
+        assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref, f"{name} h{h}")
+    # every output finite
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+DEC_CASES = [
+    # B, Lmax, L, Hq, Hkv, D, W, w0, mode, outliers
+    (1, 1024, 1000, 4, 1, 128, 300, 200, jo.MODE_SELF_EXTEND, 0.0),
+    (2, 1024, 1000, 8, 2, 128, 300, 200, jo.MODE_NONE, 0.01),
+    (1, 512, 512, 2, 1, 64, 128, 32, jo.MODE_SELF_EXTEND, 0.0),
+    (3, 5000, 4097, 8, 1, 128, 1000, 0, jo.MODE_SELF_EXTEND, 0.01),   # w0 = 0
+    (1, 700, 700, 4, 2, 128, 100, 700, jo.MODE_SELF_EXTEND, 0.0),     # plain
+    (1, 300, 1, 4, 2, 128, 100, 3, jo.MODE_SELF_EXTEND, 0.0),         # single key
+    (2, 3000, 2049, 16, 2, 64, 2048, 100, jo.MODE_SELF_EXTEND, 0.0),  # G 2 just past W, r = 8
+    (1, 20000, 19999, 6, 2, 128, 7000, 333, jo.MODE_SELF_EXTEND, 0.01),  # G 3 (64 % G != 0)
+]
+
+
+@pytest.mark.parametrize("B,Lmax,L,Hq,Hkv,D,W,w0,mode,outl", DEC_CASES)
+def test_decode_cases(B, Lmax, L, Hq, Hkv, D, W, w0, mode, outl):
+    q, kc, vc = synthetic.decode_inputs(B, Lmax, Hq, Hkv, D, seed=L, outlier_frac=outl, length=L)
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=10000.0, mode=mode)
+    o, lse, err = run_decode(q, kc, vc, L=L, w0=w0, W=W, base=10000.0, mode=mode)
+    assert err == 0
+    o_ref, lse_ref = jo.decode(q.float().numpy(), kc.float().numpy(), vc.float().numpy(), p)
+    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"decode L{L}")
+
+
+@pytest.mark.parametrize("B", [1, 8])
+def test_decode_full_size(B):
+    # Qwen3-4B shape: 32 q heads / 8 kv heads, d 128, cache of 131072 keys, G 4, w0 4096
+    L, W, w0 = 131072, 32768, 4096
+    q, kc, vc = synthetic.decode_inputs(B, L, 32, 8, 128, seed=0)
+    o, lse, err = run_decode(q, kc, vc, L=L, w0=w0, W=W, base=1e6)
+    assert err == 0
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+    bs = [0] if B == 1 else [0, 5, 7]
+    o_ref, lse_ref = jo.decode(q[bs].float().numpy(), kc[bs].float().numpy(), vc[bs].float().numpy(), p)
+    assert_close(o[bs].numpy(), o_ref, lse[bs].numpy(), lse_ref, f"decode B{B}")
+
+
+def test_decode_workspace_reuse_and_counters_reset():
+    q, kc, vc = synthetic.decode_inputs(2, 4096, 8, 2, 128, seed=11)
+    from rope_context_extension_b200 import jetlong as jl
+    ws = torch.zeros(jl.jl_decode_workspace_bytes(2, 4096, 8, 2, 128), dtype=torch.uint8, device="cuda")
+    a = run_decode(q, kc, vc, L=4096, w0=100, W=1024, base=1e6, workspace=ws)
+    b = run_decode(q, kc, vc, L=3000, w0=100, W=1024, base=1e6, workspace=ws)
+    c = run_decode(q, kc, vc, L=4096, w0=100, W=1024, base=1e6, workspace=ws)
+    assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])
+    assert not torch.equal(a[0], b[0])
+
+
+def test_decode_matches_prefill_last_row():
+    L, W, w0 = 3000, 1000, 300
+    q, k, v = synthetic.prefill_inputs(1, L, 8, 2, 128, seed=12)
+    o_pf, lse_pf, _ = run_prefill(q, k, v, w0=w0, W=W, base=1e6)
+    o_dec, lse_dec, _ = run_decode(q[:, L - 1].contiguous(), k, v, L=L, w0=w0, W=W, base=1e6)
+    assert (o_dec - o_pf[:, L - 1]).abs().max() <= 2e-2
+    assert (lse_dec - lse_pf[:, :, L - 1]).abs().max() <= 1e-3
+
+
+# ---------------------------------------------------------------------------
+# length / band sweep with 1% x8 key outliers (Qwen3-4B shape)
+# ---------------------------------------------------------------------------
+
+SWEEP_L = [16384, 32768, 32769, 49152, 100003, 131072]
+
+
+@pytest.mark.parametrize("L", SWEEP_L)
+def test_decode_sweep(L):
+    W = 32768
+    q, kc, vc = synthetic.decode_inputs(1, L, 32, 8, 128, seed=L, outlier_frac=0.01)
+    for w0 in (0, 4096, L):
+        p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+        o, lse, err = run_decode(q, kc, vc, L=L, w0=w0, W=W, base=1e6)
+        assert err == 0
+        o_ref, lse_ref = jo.decode(q.float().numpy(), kc.float().numpy(), vc.float().numpy(), p)
+        assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"decode sweep L{L} w0{w0}")
+
+
+@pytest.mark.parametrize("L", SWEEP_L)
+def test_prefill_sweep_sampled(L):
+    W = 32768
+    q, k, v = synthetic.prefill_inputs(1, L, 32, 8, 128, seed=L, outlier_frac=0.01)
+    heads = [0, 13, 31]
+    for w0 in (0, 4096, L):
+        o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6)
+        assert err == 0
+        rows = sample_rows(L, w0, 12, seed=w0)
+        p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+        ref = oracle_prefill_rows(q, k, v, rows, heads, p)
+        for h in heads:
+            o_ref, lse_ref = ref[h]
+            assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref,
+                         f"prefill sweep L{L} w0{w0} h{h}")

@@ -1,0 +1,133 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The shared library must load, export every entry point include/jl_api.h
+declares, compute the integer position algebra bit-exactly against the
+oracle, and reject bad arguments with the documented status codes before any
+device work is launched.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import jetlong_oracle as jo
+from rope_context_extension_b200 import jetlong as jl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jl_api.h")
+
+JL_OK, JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_ALIGNMENT, JL_ERR_WORKSPACE = 0, -1, -2, -3, -4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rope_context_extension_b200 import build
+    build.build()
+    return jl.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(jl_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for want in ("jl_group_size", "jl_bifocal_prefill", "jl_bifocal_decode", "jl_remote_positions",
+                 "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) == set(jl.EXPORTED_SYMBOLS)
+
+
+def test_group_size_matches_oracle(lib):
+    for L in [0, 1, 127, 128, 129, 512, 16384, 32767, 32768, 32769, 49152, 65536, 65537, 100003, 131072, 131073]:
+        for W in (1, 128, 32768):
+            assert jl.jl_group_size(L, W) == jo.group_size(L, W)
+
+
+def test_group_size_rejects_bad_args(lib):
+    g = ctypes.c_int64(0)
+    assert lib.jl_group_size(-1, 10, ctypes.byref(g)) == JL_ERR_INVALID_ARG
+    assert lib.jl_group_size(10, 0, ctypes.byref(g)) == JL_ERR_INVALID_ARG
+    assert lib.jl_group_size(10, 10, None) == JL_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("mode", [jl.JL_QSHIFT_NONE, jl.JL_QSHIFT_SELF_EXTEND])
+@pytest.mark.parametrize("L,w0,W", [(512, 32, 128), (1, 0, 5), (1000, 0, 300), (1000, 77, 300), (4096, 4096, 1000),
+                                    (131072, 4096, 32768), (100003, 4096, 32768), (32769, 0, 32768)])
+def test_remote_positions_bit_exact(lib, L, w0, W, mode):
+    q, k = jl.jl_remote_positions(L, w0, W, mode)
+    omode = jo.MODE_NONE if mode == jl.JL_QSHIFT_NONE else jo.MODE_SELF_EXTEND
+    pq, fk = jo.remote_positions(L, w0, W, omode)
+    np.testing.assert_array_equal(q, pq.astype(np.int32))
+    np.testing.assert_array_equal(k, fk.astype(np.int32))
+
+
+def test_remote_positions_rejects_bad_args(lib):
+    assert lib.jl_remote_positions(0, 0, 10, 1, None, None) == JL_ERR_INVALID_ARG
+    assert lib.jl_remote_positions(10, -1, 10, 1, None, None) == JL_ERR_INVALID_ARG
+    assert lib.jl_remote_positions(10, 0, 10, 7, None, None) == JL_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(lib):
+    assert jl.jl_prefill_workspace_bytes(1, 131072, 32, 8, 128) >= 2 * 131072 * (32 + 8) * 128
+    assert jl.jl_prefill_workspace_bytes(0, 10, 1, 1, 64) == 0
+    assert jl.jl_decode_workspace_bytes(8, 131072, 32, 8, 128) > 0
+    assert jl.jl_decode_workspace_bytes(1, 10, 3, 2, 64) == 0  # Hq % Hkv != 0
+
+
+# Fake, never dereferenced device addresses: argument checks return before any launch.
+A = 0x10000
+
+
+def _prefill(lib, q=A, k=A, v=A, o=A, lse=None, B=1, L=256, Hq=4, Hkv=2, D=128, w0=16, W=64, base=1e4, scale=0.0,
+             mode=1, ws=A, ws_bytes=1 << 40):
+    return lib.jl_bifocal_prefill(q, k, v, o, lse, B, L, Hq, Hkv, D, w0, W, base, scale, mode, ws, ws_bytes, None,
+                                  None)
+
+
+def _decode(lib, q=A, k=A, v=A, cache_len=256, o=A, lse=None, B=1, L=256, Hq=4, Hkv=2, D=128, w0=16, W=64,
+            base=1e4, scale=0.0, mode=1, ws=A, ws_bytes=1 << 40):
+    return lib.jl_bifocal_decode(q, k, v, cache_len, o, lse, B, L, Hq, Hkv, D, w0, W, base, scale, mode, ws,
+                                 ws_bytes, None, None)
+
+
+def test_prefill_argument_errors(lib):
+    assert _prefill(lib, D=96) == JL_ERR_UNSUPPORTED
+    assert _prefill(lib, Hq=3, Hkv=2) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, L=0) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, w0=-1) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, W=0) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, base=0.0) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, mode=3) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, q=None) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, o=None) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, k=A + 8) == JL_ERR_ALIGNMENT
+    assert _prefill(lib, ws=None) == JL_ERR_WORKSPACE
+    assert _prefill(lib, ws_bytes=100) == JL_ERR_WORKSPACE
+    assert _prefill(lib, ws=A + 4) == JL_ERR_ALIGNMENT
+
+
+def test_decode_argument_errors(lib):
+    assert _decode(lib, D=80) == JL_ERR_UNSUPPORTED
+    assert _decode(lib, Hq=32, Hkv=2) == JL_ERR_UNSUPPORTED  # more than 8 query heads per KV head
+    assert _decode(lib, cache_len=100) == JL_ERR_INVALID_ARG  # L beyond the cache
+    assert _decode(lib, Hq=5, Hkv=2) == JL_ERR_INVALID_ARG
+    assert _decode(lib, v=None) == JL_ERR_INVALID_ARG
+    assert _decode(lib, o=A + 2) == JL_ERR_ALIGNMENT
+    assert _decode(lib, ws=None) == JL_ERR_WORKSPACE
+    assert _decode(lib, ws_bytes=16) == JL_ERR_WORKSPACE
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.jl_status_string(code)

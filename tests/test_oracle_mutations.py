@@ -53,7 +53,7 @@ def _rotate_interleaved(x, pos, base):
 jo_rotate_orig = jo.rope_rotate
 
 
-def _scores_swapped(q_rows, q_pos, k, p):
+def _scores_swapped(q_rows, q_pos, k, p, keys=None):
     # local and remote score sets exchanged
     i = np.asarray(q_pos)
     j = np.arange(k.shape[0])
@@ -94,6 +94,8 @@ MUTATIONS = {
 @pytest.mark.parametrize("name", list(MUTATIONS))
 def test_mutation_is_caught(name, monkeypatch):
     attr, fn = MUTATIONS[name]
+    jo._CS_CACHE.clear()  # memoised angles must not hide a planted mistake
+    monkeypatch.setattr(jo, "_CS_CACHE", {})
     if attr.startswith("BifocalParams."):
         monkeypatch.setattr(jo.BifocalParams, attr.split(".")[1], fn)
     else:
