@@ -478,12 +478,14 @@ def main():
     ap.add_argument("--decode-len", type=int, default=None, help="smaller decode L (profiling runs only)")
     ap.add_argument("--decode-batch", type=int, default=None, help="decode batch (default 8)")
     args = ap.parse_args()
-    if args.prefill_len:
-        PREFILL["L"] = args.prefill_len
-        PREFILL["workload"] += f" (L={args.prefill_len}, profiling size)"
-    if args.decode_len:
-        DECODE["L"] = args.decode_len
-        DECODE["workload"] += f" (L={args.decode_len}, profiling size)"
+    # Smaller profiling sizes keep G = L / w_pretrained and w0 / L of the full workload.
+    for cfg, n in ((PREFILL, args.prefill_len), (DECODE, args.decode_len)):
+        if n:
+            f = n / cfg["L"]
+            cfg["W"] = max(1, int(round(cfg["W"] * f)))
+            cfg["w0"] = int(round(cfg["w0"] * f))
+            cfg["L"] = n
+            cfg["workload"] += f" (profiling size L={n}, w_pretrained={cfg['W']}, w0={cfg['w0']})"
     if args.decode_batch:
         DECODE["B"] = args.decode_batch
     if args.warmup < 3 and args.impl == "ours":
