@@ -156,6 +156,30 @@ int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, i
                       double rope_base, float softmax_scale, int mode, void* workspace,
                       size_t workspace_bytes, int* dev_error, void* stream);
 
+/*
+ * jl_bifocal_decode without a workspace argument, for callers that cannot
+ * allocate device memory (e.g. a plugin inside an inference engine whose
+ * device memory is wholly owned by the host framework's pool, or a serving
+ * loop that must not allocate once it runs).  The paper has no counterpart:
+ * this is an interface convenience of this library.
+ *   Same arguments, layouts, results and errors as jl_bifocal_decode, minus
+ *   the workspace.  Scratch lives in a fixed 4 MiB device array inside the
+ *   library (held on every GPU that loads the library until exit); a problem
+ *   whose decode scratch (jl_decode_workspace_bytes) exceeds 4 MiB is rejected
+ *   with JL_ERR_WORKSPACE before any launch.
+ *   All calls on a device share that array and it keeps the last call's
+ *   contents: calls that overlap on the GPU race and give wrong results, so
+ *   order them on one stream (or with events).  The ticket counters are
+ *   cleared with cudaMemsetAsync before every launch.
+ *   The first call on a device looks up the array's address (cudaGetSymbolAddress,
+ *   with that device current) and caches it; make that first call before any
+ *   stream capture.  Nothing allocates device memory.
+ * Launches one memset and one kernel.
+ */
+int jl_bifocal_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                              float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
+                              double rope_base, float softmax_scale, int mode, int* dev_error, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

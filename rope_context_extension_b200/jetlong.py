@@ -17,7 +17,7 @@ __all__ = [
     "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JetLongError", "lib", "library_path",
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
-    "EXPORTED_SYMBOLS",
+    "jl_bifocal_decode_noalloc", "EXPORTED_SYMBOLS",
 ]
 
 JL_QSHIFT_NONE = 0
@@ -25,7 +25,7 @@ JL_QSHIFT_SELF_EXTEND = 1
 EXPORTED_SYMBOLS = (
     "jl_status_string", "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes",
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
-    "jl_prefill_attention",
+    "jl_prefill_attention", "jl_bifocal_decode_noalloc",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_decode.argtypes = [c_p, c_p, c_p, c_i64, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_f,
                                     c_i, c_p, c_sz, c_p, c_p]
     L.jl_bifocal_decode.restype = c_i
+    L.jl_bifocal_decode_noalloc.argtypes = [c_p, c_p, c_p, c_i64, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d,
+                                            c_f, c_i, c_p, c_p]
+    L.jl_bifocal_decode_noalloc.restype = c_i
     _lib = L
     return L
 
@@ -200,3 +203,25 @@ def jl_bifocal_decode(q, k_cache, v_cache, o, lse, *, L: int, w0: int, w_pretrai
                                  Hkv, D, int(w0), int(w_pretrained), float(rope_base), float(softmax_scale),
                                  int(mode), _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream))
     _check(st, "jl_bifocal_decode")
+
+
+def jl_bifocal_decode_noalloc(q, k_cache, v_cache, o, lse, *, L: int, w0: int, w_pretrained: int,
+                              rope_base: float, softmax_scale: float = 0.0, mode: int = JL_QSHIFT_SELF_EXTEND,
+                              dev_error=None, stream=None):
+    """jl_bifocal_decode for callers that cannot allocate device memory: the
+    scratch is a fixed 4 MiB array inside the library (shared by every call on
+    a device; calls that overlap on the GPU race).  Same tensors as
+    jl_bifocal_decode, no workspace."""
+    import torch
+    B, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    _check_tensor(q, "q", torch.bfloat16)
+    _check_tensor(k_cache, "k_cache", torch.bfloat16)
+    _check_tensor(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
+    _check_tensor(o, "o", torch.bfloat16, (B, Hq, D))
+    if lse is not None:
+        _check_tensor(lse, "lse", torch.float32, (B, Hq))
+    st = lib().jl_bifocal_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), Lmax, _ptr(o), _ptr(lse), B,
+                                         int(L), Hq, Hkv, D, int(w0), int(w_pretrained), float(rope_base),
+                                         float(softmax_scale), int(mode), _ptr(dev_error), _stream(stream))
+    _check(st, "jl_bifocal_decode_noalloc")
