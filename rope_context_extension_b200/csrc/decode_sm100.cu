@@ -68,26 +68,61 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// (a, b) -> bf16x2 hi = round(a, b) and lo = round(a - hi_a, b - hi_b).
-__device__ __forceinline__ void split_pair_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+// Packed fp32x2 arithmetic (one instruction for two lanes of a 64-bit pair).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// bf16x2 word -> packed fp32x2 (exact)
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2_pack(bf16lo_to_f32(w), bf16hi_to_f32(w)); }
+
+// Packed pair v = (a, b) -> bf16x2 hi = round(a, b) and lo = round((a, b) - hi).
+__device__ __forceinline__ void split_f2_bf16(uint64_t v, uint32_t& hi, uint32_t& lo) {
+  float a, b;
+  f2_unpack(v, a, b);
   hi = pack_bf16x2(a, b);
-  lo = pack_bf16x2(a - bf16lo_to_f32(hi), b - bf16hi_to_f32(hi));
+  const uint64_t r = f2_sub(v, bf16x2_to_f2(hi));
+  float ra, rb;
+  f2_unpack(r, ra, rb);
+  lo = pack_bf16x2(ra, rb);
 }
 
-// Rotate the bf16 pairs (x, y) (two lanes of a bf16x2 word each) by the complex
-// factors (c0, s0), (c1, s1) and return the results as hi / lo bf16 parts.
-__device__ __forceinline__ void rot_split_bf16(uint32_t xw, uint32_t yw, float c0, float s0, float c1, float s1,
-                                               uint32_t& xh, uint32_t& xl, uint32_t& yh, uint32_t& yl) {
-  const float x0 = bf16lo_to_f32(xw), x1 = bf16hi_to_f32(xw);
-  const float y0 = bf16lo_to_f32(yw), y1 = bf16hi_to_f32(yw);
-  split_pair_bf16(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1, xh, xl);
-  split_pair_bf16(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1, yh, yl);
+// Rotate the bf16 pairs (x, y) of two adjacent RoPE pairs by the factors
+// f = (c0, c1, s0, s1) and return the results as hi / lo bf16 parts:
+// x' = x c - y s, y' = y c + x s.
+__device__ __forceinline__ void rot_split_bf16(uint32_t xw, uint32_t yw, const float4& f, uint32_t& xh, uint32_t& xl,
+                                               uint32_t& yh, uint32_t& yl) {
+  const uint64_t x = bf16x2_to_f2(xw), y = bf16x2_to_f2(yw);
+  const uint64_t c = f2_pack(f.x, f.y), sn = f2_pack(f.z, f.w);
+  const uint64_t xr = f2_sub(f2_mul(x, c), f2_mul(y, sn));
+  const uint64_t yr = f2_fma(x, sn, f2_mul(y, c));
+  split_f2_bf16(xr, xh, xl);
+  split_f2_bf16(yr, yh, yl);
 }
 
 __device__ __forceinline__ void named_sync_consumers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(168)
     bifocal_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ DecodeArgs args) {
   using C = DecCfg<D>;
@@ -146,13 +181,15 @@ __global__ void __maxnreg__(200)
       }
       double sn, cs;
       sincos(turns * args.theta[t], &sn, &cs);
-      const float2 v = make_float2((float)cs, (float)sn);
-      if (row < 16)
-        E[row * (C::kERow / 8) + t] = v;
-      else if (row < 18)
-        F[(row - 16) * H2 + t] = v;
-      else
-        Q0[(row - 18) * H2 + t] = v;
+      // E and F rows hold (c_t, c_t+1, s_t, s_t+1) for even t; Q0 rows (c_t, s_t)
+      float* dst = row < 16 ? reinterpret_cast<float*>(E) + row * (C::kERow / 4)
+                            : reinterpret_cast<float*>(F) + (row - 16) * D;
+      if (row < 18) {
+        dst[(t >> 1) * 4 + (t & 1)] = (float)cs;
+        dst[(t >> 1) * 4 + 2 + (t & 1)] = (float)sn;
+      } else {
+        Q0[(row - 18) * H2 + t] = make_float2((float)cs, (float)sn);
+      }
     }
   }
   __syncthreads();
@@ -231,30 +268,54 @@ __global__ void __maxnreg__(200)
     }
   }
 
-  float oacc[D / 8][4];
+  // O is accumulated transposed, O^T[dim][head] += V^T[dim][key] P^T[key][head]:
+  // V^T comes from ldmatrix.trans, and P^T's B fragment is exactly the score
+  // C fragment of this lane, so no shuffle is needed.  Lane holds dims
+  // 16 mt + lane/4 (+8) for heads 2 c4 and 2 c4 + 1.
+  float oacc[D / 16][4];
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+  for (int n = 0; n < D / 16; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
   float m_used = -INFINITY, l_part = 0.f;
   const float sl2 = args.scale_log2;
   bool ok = true;
 
+  // Group arithmetic of this warp's tile start j0, advanced by 64 keys per
+  // tile without divisions: j0 = qd G + rm.
+  int j0 = t_begin * kDecKeys + 16 * warp;
+  int qd = j0 / G, rm = j0 - qd * G;
+  const int q64 = kDecKeys / G, r64 = kDecKeys - q64 * G;
+  // floor(x / G) for 0 <= x < G + 16 (one multiply-high; exact there)
+  auto div_small = [&](int x) -> int {
+    return G >= 16 ? (x >= G ? 1 : 0) : (int)__umulhi((unsigned)x, args.g_magic);
+  };
+
   for (int i = 0; i < ntile; ++i) {
     const int s = i % kDecStages;
     const uint32_t ph = (uint32_t)(i / kDecStages) & 1u;
-    const int j0 = (t_begin + i) * kDecKeys + 16 * warp;
-
-    // advance q^c from the previous tile's j0 to this one
-    if (!all_local && i > 0) {
-      const int jp = j0 - kDecKeys;
-      const int fidx = ((j0 / G) - (jp / G)) - 64 / G;  // 0 or 1
-      const float2* Fr = F + fidx * H2;
+    if (i > 0) {
+      j0 += kDecKeys;
+      qd += q64;
+      rm += r64;
+      int fidx = 0;
+      if (rm >= G) {
+        rm -= G;
+        ++qd;
+        fidx = 1;
+      }
+      // advance q^c from the previous tile's j0 to this one
+      if (!all_local) {
+        const float4* Fr = reinterpret_cast<const float4*>(F) + fidx * (H2 / 2);
 #pragma unroll
-      for (int e = 0; e < C::kNT; ++e) {
-        const int t = 16 * (e >> 2) + 2 * c4 + (e & 1) + ((e & 2) ? 8 : 0);
-        const float2 f = Fr[t];
-        const float x = qre[e], y = qim[e];
-        qre[e] = x * f.x - y * f.y;
-        qim[e] = y * f.x + x * f.y;
+        for (int e = 0; e < C::kNT; e += 2) {
+          const int t = 16 * (e >> 2) + 2 * c4 + ((e & 2) ? 8 : 0);  // even
+          const float4 f = Fr[t >> 1];
+          const uint64_t c = f2_pack(f.x, f.y), sn = f2_pack(f.z, f.w);
+          const uint64_t x = f2_pack(qre[e], qre[e + 1]), y = f2_pack(qim[e], qim[e + 1]);
+          const uint64_t xr = f2_sub(f2_mul(x, c), f2_mul(y, sn));
+          const uint64_t yr = f2_fma(x, sn, f2_mul(y, c));
+          f2_unpack(xr, qre[e], qre[e + 1]);
+          f2_unpack(yr, qim[e], qim[e + 1]);
+        }
       }
     }
 
@@ -265,26 +326,24 @@ __global__ void __maxnreg__(200)
     if (j0 < L) {
       const uint32_t kst = sbase + s * C::kStageBytes;
       const uint32_t vst = kst + C::kTileBytes;
-      // class of this 16-key tile
       const bool t_local = all_local || j0 >= local_from;
       const bool t_remote = !all_local && (j0 + 15 < local_from);
 
-      float sacc[2][4];
-      float sloc[2][4];
+      float sloc[2][4], sah[2][4], sal[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) sacc[nt][k] = sloc[nt][k] = 0.f;
+        for (int k = 0; k < 4; ++k) sloc[nt][k] = sah[nt][k] = sal[nt][k] = 0.f;
 
-      // correction rows of this lane's two keys (one per 8-key n-tile)
+      // correction rows of this lane's two keys (one per 8-key n-tile):
+      // dk(j0 + u) = dk(j0) - e(u), e(u) = u - (floor((j0 + u)/G) - floor(j0/G))
       const float4* Er[2];
       if (!t_local) {
-        const int dk0 = (j0 / G) - j0;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          const int jn = j0 + 8 * nt + (lane >> 2);
-          const int e = dk0 - ((jn / G) - jn);  // 0..15
-          Er[nt] = reinterpret_cast<const float4*>(E + e * (C::kERow / 8));
+          const int u = 8 * nt + (lane >> 2);
+          const int e = u - div_small(rm + u);
+          Er[nt] = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(E) + e * (C::kERow / 4));
         }
       }
 
@@ -321,29 +380,29 @@ __global__ void __maxnreg__(200)
           // The corrected operands are carried as bf16 hi + lo pairs (about 16
           // significant bits): the query's hi part sits in M rows 0-7 and its
           // lo part in rows 8-15 (unused by the r <= 8 heads), so two products
-          // per k-step (keys hi, keys lo) give (q_hi + q_lo) . (k_hi + k_lo)
-          // once rows h and h + 8 are added.
+          // per k-step (keys hi, keys lo; separate accumulators to shorten the
+          // dependency chains) give (q_hi + q_lo) . (k_hi + k_lo) once rows
+          // h and h + 8 of both accumulators are added.
           uint32_t kah[4], kal[4], kbh[4], kbl[4];
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             const float4 f01 = Er[nt][(16 * kp + 2 * c4) >> 1];
             const float4 f23 = Er[nt][(16 * kp + 8 + 2 * c4) >> 1];
-            rot_split_bf16(klo[2 * nt], khi[2 * nt], f01.x, f01.y, f01.z, f01.w, kah[2 * nt], kal[2 * nt],
-                           kbh[2 * nt], kbl[2 * nt]);
-            rot_split_bf16(klo[2 * nt + 1], khi[2 * nt + 1], f23.x, f23.y, f23.z, f23.w, kah[2 * nt + 1],
-                           kal[2 * nt + 1], kbh[2 * nt + 1], kbl[2 * nt + 1]);
+            rot_split_bf16(klo[2 * nt], khi[2 * nt], f01, kah[2 * nt], kal[2 * nt], kbh[2 * nt], kbl[2 * nt]);
+            rot_split_bf16(klo[2 * nt + 1], khi[2 * nt + 1], f23, kah[2 * nt + 1], kal[2 * nt + 1], kbh[2 * nt + 1],
+                           kbl[2 * nt + 1]);
           }
           uint32_t alo[4], ahi[4];
-          split_pair_bf16(qre[4 * kp + 0], qre[4 * kp + 1], alo[0], alo[1]);
-          split_pair_bf16(qre[4 * kp + 2], qre[4 * kp + 3], alo[2], alo[3]);
-          split_pair_bf16(qim[4 * kp + 0], qim[4 * kp + 1], ahi[0], ahi[1]);
-          split_pair_bf16(qim[4 * kp + 2], qim[4 * kp + 3], ahi[2], ahi[3]);
+          split_f2_bf16(f2_pack(qre[4 * kp + 0], qre[4 * kp + 1]), alo[0], alo[1]);
+          split_f2_bf16(f2_pack(qre[4 * kp + 2], qre[4 * kp + 3]), alo[2], alo[3]);
+          split_f2_bf16(f2_pack(qim[4 * kp + 0], qim[4 * kp + 1]), ahi[0], ahi[1]);
+          split_f2_bf16(f2_pack(qim[4 * kp + 2], qim[4 * kp + 3]), ahi[2], ahi[3]);
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
-            mma_bf16(sacc[nt], alo, kah[2 * nt], kah[2 * nt + 1]);
-            mma_bf16(sacc[nt], alo, kal[2 * nt], kal[2 * nt + 1]);
-            mma_bf16(sacc[nt], ahi, kbh[2 * nt], kbh[2 * nt + 1]);
-            mma_bf16(sacc[nt], ahi, kbl[2 * nt], kbl[2 * nt + 1]);
+            mma_bf16(sah[nt], alo, kah[2 * nt], kah[2 * nt + 1]);
+            mma_bf16(sal[nt], alo, kal[2 * nt], kal[2 * nt + 1]);
+            mma_bf16(sah[nt], ahi, kbh[2 * nt], kbh[2 * nt + 1]);
+            mma_bf16(sal[nt], ahi, kbl[2 * nt], kbl[2 * nt + 1]);
           }
         }
       }
@@ -356,7 +415,8 @@ __global__ void __maxnreg__(200)
         for (int k = 0; k < 2; ++k) {
           const int j = j0 + 8 * nt + 2 * c4 + k;
           const bool loc = all_local || j >= local_from;
-          float v = (loc ? sloc[nt][k] : sacc[nt][k] + sacc[nt][k + 2]) * sl2;
+          const float rem = (sah[nt][k] + sah[nt][k + 2]) + (sal[nt][k] + sal[nt][k + 2]);
+          float v = (loc ? sloc[nt][k] : rem) * sl2;
           if (j >= L) v = -INFINITY;
           x[nt][k] = v;
         }
@@ -373,10 +433,15 @@ __global__ void __maxnreg__(200)
         m_used = m_new;
       }
       if (__any_sync(0xffffffffu, resc)) {
+        // this lane's O^T columns are heads 2 c4 and 2 c4 + 1
+        const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c4);
+        const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c4 + 4);
 #pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-          oacc[n][0] *= alpha;
-          oacc[n][1] *= alpha;
+        for (int n = 0; n < D / 16; ++n) {
+          oacc[n][0] *= a0;
+          oacc[n][1] *= a1;
+          oacc[n][2] *= a0;
+          oacc[n][3] *= a1;
         }
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
@@ -388,17 +453,17 @@ __global__ void __maxnreg__(200)
           p[nt][k] = ex2_approx(x[nt][k] - msub);
           l_part += p[nt][k];
         }
-      const uint32_t pa[4] = {pack_bf16x2(p[0][0], p[0][1]), 0u, pack_bf16x2(p[1][0], p[1][1]), 0u};
+      const uint32_t pb0 = pack_bf16x2(p[0][0], p[0][1]);  // keys 2 c4 + {0, 1}, head lane/4
+      const uint32_t pb1 = pack_bf16x2(p[1][0], p[1][1]);  // keys 8 + 2 c4 + {0, 1}
 #pragma unroll
-      for (int np = 0; np < D / 16; ++np) {
+      for (int mt = 0; mt < D / 16; ++mt) {
         const int mi = lane >> 3;
-        const int kr = 16 * warp + (mi & 1) * 8 + (lane & 7);
-        const int u = 2 * (np & 3) + (mi >> 1);
-        const uint32_t addr = vst + (np >> 2) * (kDecKeys * 128) + kr * 128 + ((u ^ (kr & 7)) << 4);
-        uint32_t v0, v1, v2, v3;
-        ldsm_x4_t(addr, v0, v1, v2, v3);
-        mma_bf16(oacc[2 * np], pa, v0, v1);
-        mma_bf16(oacc[2 * np + 1], pa, v2, v3);
+        const int kr = 16 * warp + (mi >> 1) * 8 + (lane & 7);
+        const int u = 2 * (mt & 3) + (mi & 1);
+        const uint32_t addr = vst + (mt >> 2) * (kDecKeys * 128) + kr * 128 + ((u ^ (kr & 7)) << 4);
+        uint32_t va[4];
+        ldsm_x4_t(addr, va[0], va[1], va[2], va[3]);
+        mma_bf16(oacc[mt], va, pb0, pb1);
       }
     }
     __syncwarp();
@@ -412,15 +477,17 @@ __global__ void __maxnreg__(200)
   float* mw = reinterpret_cast<float*>(smem);                    // [4][kMaxR]
   float* lw = mw + 4 * kMaxR;                                    // [4][kMaxR]
   float* ow = lw + 4 * kMaxR;                                    // [4][kMaxR][D]
-  if (head_ok) {
-    if (c4 == 0) {
-      mw[warp * kMaxR + hrow] = m_used;
-      lw[warp * kMaxR + hrow] = l_part;
-    }
+  if (head_ok && c4 == 0) {
+    mw[warp * kMaxR + hrow] = m_used;
+    lw[warp * kMaxR + hrow] = l_part;
+  }
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      ow[(warp * kMaxR + hrow) * D + 8 * n + 2 * c4] = oacc[n][0];
-      ow[(warp * kMaxR + hrow) * D + 8 * n + 2 * c4 + 1] = oacc[n][1];
+  for (int mt = 0; mt < D / 16; ++mt) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int h = 2 * c4 + (k & 1);
+      const int d = 16 * mt + (lane >> 2) + ((k & 2) ? 8 : 0);
+      if (h < r) ow[(warp * kMaxR + h) * D + d] = oacc[mt][k];
     }
   }
   named_sync_consumers();
@@ -481,21 +548,40 @@ __global__ void __maxnreg__(200)
   if (threadIdx.x == 0) args.counters[b * args.Hkv + g] = 0;  // ready for the next call
 }
 
+template <int D>
+cudaError_t set_decode_attrs() {
+  auto k = bifocal_decode_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<D>::kSmem);
+  if (e != cudaSuccess) return e;
+  // shared memory is the whole carve-out: two CTAs (~110 KB each) per SM
+  return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+}
+
 }  // namespace
+
+int decode_ctas_per_sm() {
+  static int cached = 0;
+  if (cached > 0) return cached;
+  int n = 0;
+  if (set_decode_attrs<128>() != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bifocal_decode_kernel<128>, kDecThreads,
+                                                    DecCfg<128>::kSmem) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  cached = n;
+  return n;
+}
 
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeArgs& a, int D,
                           cudaStream_t stream) {
   dim3 grid(a.splits, a.Hkv, a.B);
+  cudaError_t e;
   if (D == 128) {
-    auto k = bifocal_decode_kernel<128>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<128>::kSmem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kDecThreads, DecCfg<128>::kSmem, stream>>>(tm_k, tm_v, a);
+    if ((e = set_decode_attrs<128>()) != cudaSuccess) return e;
+    bifocal_decode_kernel<128><<<grid, kDecThreads, DecCfg<128>::kSmem, stream>>>(tm_k, tm_v, a);
   } else {
-    auto k = bifocal_decode_kernel<64>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<64>::kSmem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kDecThreads, DecCfg<64>::kSmem, stream>>>(tm_k, tm_v, a);
+    if ((e = set_decode_attrs<64>()) != cudaSuccess) return e;
+    bifocal_decode_kernel<64><<<grid, kDecThreads, DecCfg<64>::kSmem, stream>>>(tm_k, tm_v, a);
   }
   return cudaGetLastError();
 }

@@ -2,6 +2,7 @@
 // tensor-map encoding and kernel launches.  See include/jl_api.h.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -78,13 +79,38 @@ int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained
 
 float resolve_scale(float s, int D) { return s == 0.f ? 1.0f / std::sqrt((float)D) : s; }
 
-// Decode split count: about two CTAs per SM over all (batch, KV head) pairs.
+// Upper bound of the decode split count (sizes the scratch): two CTA waves
+// over all (batch, KV head) pairs at two CTAs per SM.  The scratch is then at
+// most about 2 * 2 * SMs * r * (D + 2) * 4 bytes (2.5 MB at r = 8, D = 128).
 int decode_splits_max(int B, int Hkv) {
-  const int target = 2 * device_sms();
-  int s = (target + B * Hkv - 1) / (B * Hkv);
+  const int slots = 2 * device_sms();
+  int s = (2 * slots + B * Hkv - 1) / (B * Hkv);
   if (s < 1) s = 1;
   if (s > 4096) s = 4096;
   return s;
+}
+
+// Split count for one call: whole 64-key tiles per split, and the CTA count
+// chosen so the last wave on the GPU is as full as possible (at least four
+// tiles per split so the per-CTA set-up stays small).
+int decode_splits(int B, int Hkv, int ntiles) {
+  const int n = B * Hkv;
+  const int slots = jl::decode_ctas_per_sm() * device_sms();
+  const int smax = std::min(decode_splits_max(B, Hkv), std::max(1, ntiles / 4));
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= smax; ++s) {
+    const long ctas = (long)n * s;
+    const long waves = (ctas + slots - 1) / slots;
+    // time ~ waves x (tiles per split) + a small per-split overhead
+    const double per = (double)((ntiles + s - 1) / s) + 2.0;
+    const double cost = (double)waves * per;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 struct DecodeLayout {
@@ -286,8 +312,7 @@ int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, i
       (lse && ((uintptr_t)lse & 3u)))
     return JL_ERR_ALIGNMENT;
   const int ntiles = (L + 63) / 64;
-  int splits = decode_splits_max(B, Hkv);
-  if (splits > ntiles) splits = ntiles;
+  const int splits = decode_splits(B, Hkv, ntiles);
   const DecodeLayout lay = decode_layout(B, Hq, Hkv, D, decode_splits_max(B, Hkv));
   if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
@@ -321,6 +346,7 @@ int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, i
   a.w0 = all_local ? (1 << 30) : w0;
   a.all_local = all_local ? 1 : 0;
   a.G = G;
+  a.g_magic = G < 16 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)G - 1) / (uint64_t)G) : 0u;
   a.dq = jl::query_remote(L - 1, G, shift) - (L - 1);
   a.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
   fill_theta(a.theta, D, rope_base);

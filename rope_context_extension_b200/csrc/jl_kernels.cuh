@@ -48,11 +48,14 @@ struct DecodeArgs {
   int splits, ntiles;      // 64-key tiles in [0, L)
   int w0, all_local;
   int64_t G;
+  uint32_t g_magic;        // ceil(2^32 / G) for G < 16 (floor(x / G) = umulhi(x, g_magic), x < 32)
   int64_t dq;              // p_q(L - 1) - (L - 1)
   float scale_log2;
   double theta[kMaxHalfDim];
 };
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeArgs& a, int D,
                           cudaStream_t stream);
+// Resident decode CTAs per SM (occupancy of the D = 128 kernel, cached).
+int decode_ctas_per_sm();
 
 }  // namespace jl
