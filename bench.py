@@ -214,15 +214,17 @@ def run_ours(args):
 
     pkw = dict(w0=P["w0"], w_pretrained=P["W"], stream=stream)
 
-    def prefill_step(evs=None, w0=None):
+    def prefill_step(evs=None, w0=None, mode=jl.JL_QSHIFT_SELF_EXTEND, wsp=None):
         w = P["w0"] if w0 is None else w0
+        wsb = ws if wsp is None else wsp
         if evs:
             evs[0].record(stream)
-        jl.jl_prefill_correction(q, k, w0=w, w_pretrained=P["W"], rope_base=P["base"], workspace=ws, stream=stream)
+        jl.jl_prefill_correction(q, k, w0=w, w_pretrained=P["W"], rope_base=P["base"], mode=mode, workspace=wsb,
+                                 stream=stream)
         if evs:
             evs[1].record(stream)
-        jl.jl_prefill_attention(q, k, v, o, lse, w0=w, w_pretrained=P["W"], workspace=ws, dev_error=err,
-                                stream=stream)
+        jl.jl_prefill_attention(q, k, v, o, lse, w0=w, w_pretrained=P["W"], mode=mode, workspace=wsb,
+                                dev_error=err, stream=stream)
         if evs:
             evs[2].record(stream)
 
@@ -292,6 +294,13 @@ def run_ours(args):
 
     plain_pre_ms = time_calls(lambda: prefill_step(w0=P["L"]), max(2, K // 2))
     plain_dec_ms = time_calls(lambda: decode_step(w0=Dc["L"]), max(2, K // 2))
+    # split-precision remote products (for inputs with dominant large-norm keys)
+    split_pre_ms = None
+    if not args.no_split:
+        ws2 = torch.empty(2 * ws.numel(), dtype=torch.uint8, device=dev)
+        split_pre_ms = time_calls(lambda: prefill_step(mode=jl.JL_QSHIFT_SELF_EXTEND | jl.JL_REMOTE_SPLIT, wsp=ws2),
+                                  2)
+        del ws2
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -359,6 +368,8 @@ def run_ours(args):
                                     "frac": round(dec_gbs_kernel / peaks["hbm_gbs"], 4),
                                     "traffic": traffic.get("decode", {}).get("bytes_per_launch"),
                                     "peak_source": f"{peak_kind} hbm_gbs"}},
+            "prefill_split_precision": None if split_pre_ms is None else {
+                "ms": round(split_pre_ms, 3), "tflops": round(flop / (split_pre_ms * 1e-3) / 1e12, 2)},
             "plain_rope_same_kernels": {
                 "prefill_ms": round(plain_pre_ms, 3),
                 "prefill_tflops": round(flop / (plain_pre_ms * 1e-3) / 1e12, 2),
@@ -472,6 +483,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-split", action="store_true", help="skip the split-precision prefill measurement")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=4)
     ap.add_argument("--prefill-len", type=int, default=None, help="smaller prefill L (profiling runs only)")

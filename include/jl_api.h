@@ -60,6 +60,17 @@ typedef enum {
 
 typedef enum { JL_QSHIFT_NONE = 0, JL_QSHIFT_SELF_EXTEND = 1 } jl_qshift;
 
+/*
+ * Optional flag OR-ed into `mode` of the prefill and decode entry points.
+ * JL_REMOTE_SPLIT: prefill forms remote scores from fp16 hi + lo corrected rows
+ * (Q_hi K_hi + Q_hi K_lo + Q_lo K_hi, about 2^-21 relative operand error
+ * instead of 2^-12), for inputs where a few keys of large norm dominate the
+ * softmax and the fp16 rounding of the default path shows in the LSE.  It runs
+ * one query head per CTA and needs twice the prefill workspace.  Decode always
+ * carries its corrected operands as hi + lo pairs and ignores the flag.
+ */
+enum { JL_REMOTE_SPLIT = 2 };
+
 /* Human-readable name of a status code (static string). */
 const char* jl_status_string(int status);
 
@@ -82,7 +93,8 @@ int jl_remote_positions(int64_t L, int64_t w0, int64_t w_pretrained, int mode, i
 
 /*
  * Scratch bytes jl_bifocal_prefill needs: space for the remote-rotated Q and K
- * rows (2 * B * L * (Hq + Hkv) * D bytes plus alignment).  0 on bad arguments.
+ * rows (2 * B * L * (Hq + Hkv) * D bytes plus alignment); twice this with
+ * JL_REMOTE_SPLIT in `mode`.  0 on bad arguments.
  */
 size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim);
 

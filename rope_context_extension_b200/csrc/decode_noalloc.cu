@@ -62,7 +62,7 @@ extern "C" int jl_bifocal_decode_noalloc(const void* q, const void* k_cache, con
   // error launches nothing here either (not even the counter clear).
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || w0 < 0 || w_pretrained < 1 || Hq % Hkv != 0)
     return JL_ERR_INVALID_ARG;
-  if (!(rope_base > 0.0) || (mode != JL_QSHIFT_NONE && mode != JL_QSHIFT_SELF_EXTEND)) return JL_ERR_INVALID_ARG;
+  if (!(rope_base > 0.0) || (mode & ~(JL_QSHIFT_SELF_EXTEND | JL_REMOTE_SPLIT)) != 0) return JL_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return JL_ERR_UNSUPPORTED;
   if (Hq / Hkv > 8 || L > (1 << 30)) return JL_ERR_UNSUPPORTED;
   if (!q || !k_cache || !v_cache || !o || cache_len < L || cache_len > ((int64_t)1 << 31)) return JL_ERR_INVALID_ARG;

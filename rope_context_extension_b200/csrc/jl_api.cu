@@ -70,7 +70,7 @@ void fill_theta(double* theta, int D, double base) {
 int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained, double rope_base, int mode) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || w0 < 0 || w_pretrained < 1) return JL_ERR_INVALID_ARG;
   if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return JL_ERR_INVALID_ARG;
-  if (mode != JL_QSHIFT_NONE && mode != JL_QSHIFT_SELF_EXTEND) return JL_ERR_INVALID_ARG;
+  if ((mode & ~(JL_QSHIFT_SELF_EXTEND | JL_REMOTE_SPLIT)) != 0) return JL_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
   if (L > (1 << 30)) return JL_ERR_UNSUPPORTED;
@@ -195,19 +195,23 @@ int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, in
   if (st != JL_OK) return st;
   const int64_t G = jl::group_size(L, w_pretrained);
   if (jl::all_local(L, w0, G)) return JL_OK;  // nothing to correct
-  if (!workspace || workspace_bytes < jl_prefill_workspace_bytes(B, L, Hq, Hkv, D)) return JL_ERR_WORKSPACE;
+  const bool split = (mode & JL_REMOTE_SPLIT) != 0;
+  const size_t base_bytes = jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
+  if (!workspace || workspace_bytes < (split ? 2 : 1) * base_bytes) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* lo_base = reinterpret_cast<char*>(workspace) + base_bytes;  // split: Q_lo then K_lo
   RotateArgs ra;
   std::memset(&ra, 0, sizeof(ra));
   fill_theta(ra.theta, D, rope_base);
   ra.G = G;
-  ra.shift = jl::query_shift(w0, G, mode);
+  ra.shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
   ra.B = B;
   ra.L = L;
   // queries that have a remote key: i >= w0
   ra.x = reinterpret_cast<const __nv_bfloat16*>(q);
   ra.y = q_rem_ptr(workspace);
+  ra.y_lo = split ? q_rem_ptr(lo_base) : nullptr;
   ra.H = Hq;
   ra.row_begin = w0;
   ra.row_end = L;
@@ -216,6 +220,7 @@ int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, in
   // keys that have a remote query: j <= L - 1 - w0
   ra.x = reinterpret_cast<const __nv_bfloat16*>(k);
   ra.y = k_rem_ptr(workspace, B, L, Hq, D);
+  ra.y_lo = split ? k_rem_ptr(lo_base, B, L, Hq, D) : nullptr;
   ra.H = Hkv;
   ra.row_begin = 0;
   ra.row_end = L - w0;
@@ -234,11 +239,13 @@ int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, f
   if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
   const int64_t G = jl::group_size(L, w_pretrained);
   const bool all_local = jl::all_local(L, w0, G);
+  const bool split = !all_local && (mode & JL_REMOTE_SPLIT) != 0;
+  const size_t base_bytes = jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
   if (!all_local) {
-    if (!workspace || workspace_bytes < jl_prefill_workspace_bytes(B, L, Hq, Hkv, D)) return JL_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < (split ? 2 : 1) * base_bytes) return JL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
   }
-  CUtensorMap tq, tqr, tk, tkr, tv;
+  CUtensorMap tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo;
   if (!encode_bf16_4d(&tq, q, D, Hq, L, B, 128) || !encode_bf16_4d(&tk, k, D, Hkv, L, B, 128) ||
       !encode_bf16_4d(&tv, v, D, Hkv, L, B, 128))
     return JL_ERR_CUDA;
@@ -251,6 +258,15 @@ int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, f
     tqr = tq;
     tkr = tk;
   }
+  if (split) {
+    void* lo = reinterpret_cast<char*>(const_cast<void*>(workspace)) + base_bytes;
+    if (!encode_f16_4d(&tqr_lo, q_rem_ptr(lo), D, Hq, L, B, 128) ||
+        !encode_f16_4d(&tkr_lo, k_rem_ptr(lo, B, L, Hq, D), D, Hkv, L, B, 128))
+      return JL_ERR_CUDA;
+  } else {
+    tqr_lo = tqr;
+    tkr_lo = tkr;
+  }
   const int r = Hq / Hkv;
   PrefillArgs pa;
   std::memset(&pa, 0, sizeof(pa));
@@ -262,12 +278,13 @@ int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, f
   pa.Hq = Hq;
   pa.Hkv = Hkv;
   pa.r = r;
-  pa.nh = (r % 2 == 0) ? 2 : 1;
+  pa.nh = (!split && r % 2 == 0) ? 2 : 1;
   pa.num_mb = (L + 127) / 128;
   pa.all_local = all_local ? 1 : 0;
   pa.w0 = all_local ? (1 << 30) : w0;
   pa.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
-  if (jl::launch_prefill(tq, tqr, tk, tkr, tv, pa, D, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (jl::launch_prefill(tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo, pa, D, split,
+                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return JL_ERR_CUDA;
   return JL_OK;
 }
@@ -283,7 +300,8 @@ int jl_bifocal_prefill(const void* q, const void* k, const void* v, void* o, flo
   if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
   const int64_t G = jl::group_size(L, w_pretrained);
   if (!jl::all_local(L, w0, G)) {
-    if (!workspace || workspace_bytes < jl_prefill_workspace_bytes(B, L, Hq, Hkv, D)) return JL_ERR_WORKSPACE;
+    const size_t need = ((mode & JL_REMOTE_SPLIT) ? 2 : 1) * jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
+    if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
   }
   st = jl_prefill_correction(q, k, B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode, workspace,
@@ -319,7 +337,7 @@ int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, i
 
   const int64_t G = jl::group_size(L, w_pretrained);
   const bool all_local = jl::all_local(L, w0, G);
-  const int64_t shift = jl::query_shift(w0, G, mode);
+  const int64_t shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
 
   CUtensorMap tk, tv;
   if (!encode_bf16_4d(&tk, k_cache, D, Hkv, cache_len, B, 64) ||

@@ -10,7 +10,8 @@ constexpr int kMaxHalfDim = 64;  // head_dim <= 128
 // Correction rotation of rows [row_begin, row_end) of a [B, L, H, D] bf16 tensor.
 struct RotateArgs {
   const __nv_bfloat16* x;
-  __half* y;  // fp16 output
+  __half* y;     // fp16 output
+  __half* y_lo;  // optional fp16 residual (y + y_lo carries about 22 bits), or null
   int B, L, H;
   int row_begin, row_end;
   int is_query;      // 1: rotate by p_q(i) - i, 0: by f(j) - j
@@ -32,8 +33,9 @@ struct PrefillArgs {
   float scale_log2;  // softmax scale * log2(e)
 };
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
-                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const PrefillArgs& a,
-                           int D, cudaStream_t stream);
+                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
+                           const CUtensorMap& tm_kr_lo, const PrefillArgs& a, int D, bool split,
+                           cudaStream_t stream);
 
 // Split-KV bifocal decode (mma.sync tiles, in-register correction of keys).
 struct DecodeArgs {

@@ -23,6 +23,10 @@
 //   warps 8-11  softmax for head 1
 // TMEM columns: S_h at 128 h, O_h at 128 NH + D h.  P (bf16) overwrites the
 // first 64 columns of S_h and is the A operand of O_h += P V from TMEM.
+// Split mode (opt-in, for inputs with large-norm keys): the corrected rows
+// come as fp16 hi + lo pairs and a remote S accumulates Q_hi K_hi + Q_hi K_lo
+// + Q_lo K_hi (about 2^-21 relative error instead of 2^-12), one query head per
+// CTA so that Q_hi / Q_lo and K_hi / K_lo fit in shared memory.
 // Per pass the MMA order is S0(i), PV1(i-1), S1(i), PV0(i): each softmax group
 // works on its S while the tensor core runs the other head's two products.
 #include "jl_kernels.cuh"
@@ -37,14 +41,19 @@ constexpr int kStages = 2;
 constexpr int kThreads = 384;
 constexpr int kChunkBytes = 128 * 128;  // one 128-row x 128-byte swizzled slab
 
-template <int D>
+// kSplit: remote scores from fp16 hi + lo corrected rows (one query head per
+// CTA; the Q region holds Q_hi and Q_lo, each K stage K_hi and K_lo, and V is
+// single-buffered to fit shared memory).
+template <int D, bool kSplit>
 struct Cfg {
   static constexpr int kChunks = D / 64;  // 64-element (128 B) slabs per row
   static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kKSlots = kSplit ? 2 : 1;   // tiles per K stage
+  static constexpr int kVStages = kSplit ? 1 : kStages;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kKSlots * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   static constexpr int kUsed = kBarOff + 256;
   // Ask for enough shared memory that only one CTA fits per SM: each CTA
   // allocates up to 512 TMEM columns.
@@ -100,12 +109,13 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-template <int D>
+template <int D, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
-                           const __grid_constant__ CUtensorMap tm_v, const PrefillArgs args) {
-  using C = Cfg<D>;
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qr_lo,
+                           const __grid_constant__ CUtensorMap tm_kr_lo, const PrefillArgs args) {
+  using C = Cfg<D, kSplit>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -130,6 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(kKFull + s), 1);
       mbar_init(bar(kKEmpty + s), 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(bar(kVFull + s), 1);
       mbar_init(bar(kVEmpty + s), 1);
     }
@@ -163,39 +175,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_kr);
       tma_prefetch_map(&tm_v);
-      const uint32_t q_bytes = (uint32_t)(NH * C::kTileBytes);
-      auto load_q = [&](const CUtensorMap* m) {
-        mbar_arrive_expect_tx(bar(kQFull), q_bytes);
+      if (kSplit) {
+        tma_prefetch_map(&tm_qr_lo);
+        tma_prefetch_map(&tm_kr_lo);
+      }
+      // Q region: one tile per head (NH heads), or Q_hi / Q_lo of the single
+      // head for remote passes in split mode.
+      auto load_q = [&](bool remote) {
+        if (kSplit && remote) {
+          mbar_arrive_expect_tx(bar(kQFull), (uint32_t)(2 * C::kTileBytes));
+          for (int c = 0; c < C::kChunks; ++c) {
+            tma_load_4d(sbase + C::kQOff + c * kChunkBytes, &tm_qr, bar(kQFull), c * 64, hq0, mb * kBM, b);
+            tma_load_4d(sbase + C::kQOff + C::kTileBytes + c * kChunkBytes, &tm_qr_lo, bar(kQFull), c * 64, hq0,
+                        mb * kBM, b);
+          }
+          return;
+        }
+        const CUtensorMap* m = remote ? &tm_qr : &tm_q;
+        mbar_arrive_expect_tx(bar(kQFull), (uint32_t)(NH * C::kTileBytes));
         for (int hh = 0; hh < NH; ++hh)
           for (int c = 0; c < C::kChunks; ++c)
             tma_load_4d(sbase + C::kQOff + hh * C::kTileBytes + c * kChunkBytes, m, bar(kQFull), c * 64,
                         hq0 + hh, mb * kBM, b);
       };
-      load_q(sc.n_loc > 0 ? &tm_q : &tm_qr);
+      load_q(sc.n_loc == 0);
       int q_loads = 1;
       int k_last = -1, v_last = -1;  // last passes whose K / V copies were issued
       bool ok = true;
       for (int p = 0; p < npass; ++p) {
         const int s = p % kStages;
         const uint32_t ph = (uint32_t)(p / kStages) & 1u;
+        const int sv = p % C::kVStages;
+        const uint32_t phv = (uint32_t)(p / C::kVStages) & 1u;
         const bool remote = p >= sc.n_loc;
         const int a = remote ? sc.a_min + (p - sc.n_loc) : p;
         const int nb = mb - a;
         if (q_switch && p == sc.n_loc) {
           if (!(ok = mbar_wait(bar(kQEmpty), 0, abort_flag, args.dev_error))) break;
-          load_q(&tm_qr);
+          load_q(true);
           ++q_loads;
         }
         if (!(ok = mbar_wait(bar(kKEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
-        mbar_arrive_expect_tx(bar(kKFull + s), (uint32_t)C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sbase + C::kKOff + s * C::kTileBytes + c * kChunkBytes, remote ? &tm_kr : &tm_k,
-                      bar(kKFull + s), c * 64, kvh, nb * kBN, b);
+        const uint32_t kdst = sbase + C::kKOff + s * C::kKSlots * C::kTileBytes;
+        const bool two = kSplit && remote;
+        mbar_arrive_expect_tx(bar(kKFull + s), (uint32_t)((two ? 2 : 1) * C::kTileBytes));
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_4d(kdst + c * kChunkBytes, remote ? &tm_kr : &tm_k, bar(kKFull + s), c * 64, kvh, nb * kBN, b);
+          if (two)
+            tma_load_4d(kdst + C::kTileBytes + c * kChunkBytes, &tm_kr_lo, bar(kKFull + s), c * 64, kvh, nb * kBN,
+                        b);
+        }
         k_last = p;
-        if (!(ok = mbar_wait(bar(kVEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
-        mbar_arrive_expect_tx(bar(kVFull + s), (uint32_t)C::kTileBytes);
+        if (!(ok = mbar_wait(bar(kVEmpty + sv), phv ^ 1u, abort_flag, args.dev_error))) break;
+        mbar_arrive_expect_tx(bar(kVFull + sv), (uint32_t)C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sbase + C::kVOff + s * C::kTileBytes + c * kChunkBytes, &tm_v, bar(kVFull + s), c * 64,
+          tma_load_4d(sbase + C::kVOff + sv * C::kTileBytes + c * kChunkBytes, &tm_v, bar(kVFull + sv), c * 64,
                       kvh, nb * kBN, b);
         v_last = p;
       }
@@ -204,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(kQFull), (uint32_t)(q_loads - 1) & 1u);
         for (int p = max(0, k_last - kStages + 1); p <= k_last; ++p)
           drain_wait(bar(kKFull + p % kStages), (uint32_t)(p / kStages) & 1u);
-        for (int p = max(0, v_last - kStages + 1); p <= v_last; ++p)
-          drain_wait(bar(kVFull + p % kStages), (uint32_t)(p / kStages) & 1u);
+        for (int p = max(0, v_last - C::kVStages + 1); p <= v_last; ++p)
+          drain_wait(bar(kVFull + p % C::kVStages), (uint32_t)(p / C::kVStages) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -227,13 +261,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         const uint32_t qa = sbase + C::kQOff + h * C::kTileBytes;
-        const uint32_t ka = sbase + C::kKOff + s * C::kTileBytes;
-        const uint32_t id_s = p >= sc.n_loc ? id_s_rem : id_s_loc;
+        const uint32_t ka = sbase + C::kKOff + s * C::kKSlots * C::kTileBytes;
+        const bool remote = p >= sc.n_loc;
+        const uint32_t id_s = remote ? id_s_rem : id_s_loc;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
           mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
                  id_s, ks > 0 ? 1u : 0u);
+        }
+        if (kSplit && remote) {
+          // + Q_hi K_lo + Q_lo K_hi into the same accumulator
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
+            mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + off, 16, 1024),
+                   make_sdesc_sw128(ka + C::kTileBytes + off, 16, 1024), id_s, 1u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
+            mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + C::kTileBytes + off, 16, 1024),
+                   make_sdesc_sw128(ka + off, 16, 1024), id_s, 1u);
+          }
         }
         tc_commit(bar(kSFull + h));
         if (h == NH - 1) {
@@ -243,8 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto issue_pv = [&](int h, int p) -> bool {
-        const int s = p % kStages;
-        const uint32_t ph = (uint32_t)(p / kStages) & 1u;
+        const int s = p % C::kVStages;
+        const uint32_t ph = (uint32_t)(p / C::kVStages) & 1u;
         if (h == 0 && !mbar_wait(bar(kVFull + s), ph, abort_flag, args.dev_error)) return false;
         if (!mbar_wait(bar(kPFull + h), (uint32_t)p & 1u, abort_flag, args.dev_error)) return false;
         tc_fence_after();
@@ -414,24 +464,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
+template <int D, bool kSplit>
+cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
+                             const CUtensorMap& tm_kr_lo, const PrefillArgs& a, cudaStream_t stream) {
+  auto k = bifocal_prefill_kernel<D, kSplit>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, kSplit>::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.Hq / a.nh, a.num_mb, a.B);
+  k<<<grid, kThreads, Cfg<D, kSplit>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
-                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const PrefillArgs& a,
-                           int D, cudaStream_t stream) {
-  dim3 grid(a.Hq / a.nh, a.num_mb, a.B);
-  if (D == 128) {
-    auto k = bifocal_prefill_kernel<128>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<128>::kSmem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, Cfg<128>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, a);
-  } else {
-    auto k = bifocal_prefill_kernel<64>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<64>::kSmem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, Cfg<64>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, a);
-  }
-  return cudaGetLastError();
+                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
+                           const CUtensorMap& tm_kr_lo, const PrefillArgs& a, int D, bool split,
+                           cudaStream_t stream) {
+  if (D == 128)
+    return split ? launch_prefill_t<128, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
+                 : launch_prefill_t<128, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
+  return split ? launch_prefill_t<64, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
+               : launch_prefill_t<64, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
 }
 
 }  // namespace jl

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kRotThreads)
     const uint4 hi = *reinterpret_cast<const uint4*>(args.x + base + H2 + ch * 8);
     const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w};
     const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w};
-    uint32_t lo_out[4], hi_out[4];
+    float rx[8], ry[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float2 c0 = cs[r][ch * 8 + 2 * k];
@@ -68,12 +68,33 @@ __global__ void __launch_bounds__(kRotThreads)
       const float x0 = bf16lo_to_f32(lw[k]), x1 = bf16hi_to_f32(lw[k]);
       const float y0 = bf16lo_to_f32(hw[k]), y1 = bf16hi_to_f32(hw[k]);
       // (x, y) -> (x cos - y sin, y cos + x sin)
-      lo_out[k] = pack_f16x2(x0 * c0.x - y0 * c0.y, x1 * c1.x - y1 * c1.y);
-      hi_out[k] = pack_f16x2(y0 * c0.x + x0 * c0.y, y1 * c1.x + x1 * c1.y);
+      rx[2 * k] = x0 * c0.x - y0 * c0.y;
+      rx[2 * k + 1] = x1 * c1.x - y1 * c1.y;
+      ry[2 * k] = y0 * c0.x + x0 * c0.y;
+      ry[2 * k + 1] = y1 * c1.x + x1 * c1.y;
+    }
+    uint32_t lo_out[4], hi_out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      lo_out[k] = pack_f16x2(rx[2 * k], rx[2 * k + 1]);
+      hi_out[k] = pack_f16x2(ry[2 * k], ry[2 * k + 1]);
     }
     *reinterpret_cast<uint4*>(args.y + base + ch * 8) = make_uint4(lo_out[0], lo_out[1], lo_out[2], lo_out[3]);
     *reinterpret_cast<uint4*>(args.y + base + H2 + ch * 8) =
         make_uint4(hi_out[0], hi_out[1], hi_out[2], hi_out[3]);
+    if (args.y_lo != nullptr) {
+      // residuals of the fp16 rounding, themselves rounded to fp16
+      uint32_t rl[4], rh[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __half2 a = *reinterpret_cast<const __half2*>(&lo_out[k]);
+        const __half2 c = *reinterpret_cast<const __half2*>(&hi_out[k]);
+        rl[k] = pack_f16x2(rx[2 * k] - __low2float(a), rx[2 * k + 1] - __high2float(a));
+        rh[k] = pack_f16x2(ry[2 * k] - __low2float(c), ry[2 * k + 1] - __high2float(c));
+      }
+      *reinterpret_cast<uint4*>(args.y_lo + base + ch * 8) = make_uint4(rl[0], rl[1], rl[2], rl[3]);
+      *reinterpret_cast<uint4*>(args.y_lo + base + H2 + ch * 8) = make_uint4(rh[0], rh[1], rh[2], rh[3]);
+    }
   }
 }
 

@@ -14,7 +14,7 @@ import os
 import numpy as np
 
 __all__ = [
-    "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JetLongError", "lib", "library_path",
+    "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JL_REMOTE_SPLIT", "JetLongError", "lib", "library_path",
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "EXPORTED_SYMBOLS",
@@ -22,6 +22,7 @@ __all__ = [
 
 JL_QSHIFT_NONE = 0
 JL_QSHIFT_SELF_EXTEND = 1
+JL_REMOTE_SPLIT = 2  # OR into mode: fp16 hi + lo remote operands in prefill (twice the workspace)
 EXPORTED_SYMBOLS = (
     "jl_status_string", "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes",
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",

@@ -12,7 +12,8 @@ import torch
 
 from oracle import jetlong_oracle as jo
 from rope_context_extension_b200 import synthetic
-from tests.gpu_helpers import (assert_close, oracle_prefill_rows, run_decode, run_prefill, sample_rows)
+from tests.gpu_helpers import (LSE_MAX_ABS, LSE_MAX_ABS_FP16_OUTLIERS, assert_close, oracle_prefill_rows,
+                               run_decode, run_prefill, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -53,14 +54,16 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("B,L,Hq,Hkv,D,W,w0,mode,outl", CASES)
-def test_prefill_small_cases(B, L, Hq, Hkv, D, W, w0, mode, outl):
+def test_prefill_small_cases(B, L, Hq, Hkv, D, W, w0, mode, outl, split):
     q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=L + w0, outlier_frac=outl)
     p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=10000.0, mode=mode)
-    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=10000.0, mode=mode)
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=10000.0, mode=mode, split=split)
     assert err == 0
     o_ref, lse_ref = jo.prefill_dense(q.float().numpy(), k.float().numpy(), v.float().numpy(), p)
-    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"L{L} w0{w0}")
+    tol = LSE_MAX_ABS if (split or outl == 0.0) else LSE_MAX_ABS_FP16_OUTLIERS
+    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"L{L} w0{w0} split{split}", lse_tol=tol)
 
 
 def test_prefill_plain_mode_is_identical_across_equivalent_calls():
@@ -184,13 +187,14 @@ def test_decode_sweep(L):
         assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"decode sweep L{L} w0{w0}")
 
 
+@pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("L", SWEEP_L)
-def test_prefill_sweep_sampled(L):
+def test_prefill_sweep_sampled(L, split):
     W = 32768
     q, k, v = synthetic.prefill_inputs(1, L, 32, 8, 128, seed=L, outlier_frac=0.01)
     heads = [0, 13, 31]
     for w0 in (0, 4096, L):
-        o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6)
+        o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6, split=split)
         assert err == 0
         rows = sample_rows(L, w0, 12, seed=w0)
         p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
@@ -198,4 +202,20 @@ def test_prefill_sweep_sampled(L):
         for h in heads:
             o_ref, lse_ref = ref[h]
             assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref,
-                         f"prefill sweep L{L} w0{w0} h{h}")
+                         f"prefill sweep L{L} w0{w0} h{h} split{split}",
+                         lse_tol=LSE_MAX_ABS if split else LSE_MAX_ABS_FP16_OUTLIERS)
+
+
+def test_prefill_split_mode_full_size_sampled():
+    # the Qwen3-8B-shaped 128K workload through the split-precision path
+    L, W, w0 = 131072, 32768, 4096
+    q, k, v = synthetic.prefill_inputs(1, L, 32, 8, 128, seed=0)
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6, split=True)
+    assert err == 0
+    rows = sample_rows(L, w0, 24, seed=2)
+    heads = [0, 17, 31]
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+    ref = oracle_prefill_rows(q, k, v, rows, heads, p)
+    for h in heads:
+        o_ref, lse_ref = ref[h]
+        assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref, f"split 128k h{h}")

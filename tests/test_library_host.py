@@ -76,6 +76,7 @@ def test_remote_positions_rejects_bad_args(lib):
     assert lib.jl_remote_positions(0, 0, 10, 1, None, None) == JL_ERR_INVALID_ARG
     assert lib.jl_remote_positions(10, -1, 10, 1, None, None) == JL_ERR_INVALID_ARG
     assert lib.jl_remote_positions(10, 0, 10, 7, None, None) == JL_ERR_INVALID_ARG
+    assert lib.jl_remote_positions(10, 0, 10, 2, None, None) == JL_ERR_INVALID_ARG  # not a position-map mode
 
 
 def test_workspace_sizes(lib):
@@ -108,7 +109,10 @@ def test_prefill_argument_errors(lib):
     assert _prefill(lib, w0=-1) == JL_ERR_INVALID_ARG
     assert _prefill(lib, W=0) == JL_ERR_INVALID_ARG
     assert _prefill(lib, base=0.0) == JL_ERR_INVALID_ARG
-    assert _prefill(lib, mode=3) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, mode=4) == JL_ERR_INVALID_ARG
+    # split precision (mode bit 2) needs twice the workspace
+    need = lib.jl_prefill_workspace_bytes(1, 256, 4, 2, 128)
+    assert _prefill(lib, mode=3, ws_bytes=need) == JL_ERR_WORKSPACE
     assert _prefill(lib, q=None) == JL_ERR_INVALID_ARG
     assert _prefill(lib, o=None) == JL_ERR_INVALID_ARG
     assert _prefill(lib, k=A + 8) == JL_ERR_ALIGNMENT
