@@ -39,6 +39,10 @@ constexpr int kBM = 128;  // query rows per block
 constexpr int kBN = 128;  // keys per tile
 constexpr int kStages = 2;
 constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
+constexpr int kLowRegs = 104;      // warpgroup 0: TMA producer, MMA issuer
+constexpr int kHighRegs = 200;    // warpgroups 1-2: softmax
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kChunkBytes = 128 * 128;  // one 128-row x 128-byte swizzled slab
 
 // kSplit: remote scores from fp16 hi + lo corrected rows (one query head per
@@ -162,11 +166,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+
   const Sched sc = make_sched(mb, args.w0, args.all_local != 0);
   const int npass = sc.n_loc + sc.n_rem;
   const bool q_switch = sc.n_loc > 0 && sc.n_rem > 0;
   const int w0 = args.w0;
 
+  // Register split: the producer / MMA warpgroup needs few registers, the two
+  // softmax warpgroups hold a 128-column score row each.  The launch gives
+  // 384 x kLaunchRegs; 128 x kLowRegs + 256 x kHighRegs stays within it (the
+  // host refuses to launch if the compiled register count differs).  Each
+  // warpgroup changes its budget once, at the top of its own branch.
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -331,7 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(kDrain), 0);
       }
     }
-  } else if (warp >= 4 && ((warp - 4) >> 2) < NH) {
+  }
+  } else {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+  if (((warp - 4) >> 2) < NH) {
     // ------------------------------------------------------------ softmax
     const int h = (warp - 4) >> 2;
     const int wq = warp & 3;
@@ -359,11 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
 
-      float x[128];
+      float x[128];  // raw scores (fp32 accumulator values)
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]) * sl2;
+        for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]);
 
       const bool need_mask = remote ? (128 * a - 127 < w0) : (a == 0 || 128 * a + 127 >= w0);
       if (need_mask) {
@@ -375,9 +390,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!keep) x[col] = -INFINITY;
         }
       }
-      float mt = x[0];
+      // Row max over four independent chains of three-input maxima (the scale
+      // is positive, so the max of the raw scores scales to the max of the
+      // scaled ones).
+      float m4[4];
 #pragma unroll
-      for (int col = 1; col < 128; ++col) mt = fmaxf(mt, x[col]);
+      for (int j = 0; j < 4; ++j) m4[j] = fmaxf(x[j], x[4 + j]);
+#pragma unroll
+      for (int col = 8; col < 128; col += 8)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m4[j] = fmax3(m4[j], x[col + j], x[col + 4 + j]);
+      const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
       const float m_new = fmaxf(m_used, mt);
       float alpha = 1.f;
       bool rescale_o = false;
@@ -395,20 +418,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
 
-      float rs = 0.f;
+      // p = 2^(s * scale * log2 e - m): one packed FMA per pair, the row sum in
+      // two packed accumulators.
+      const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-msub, -msub);
+      uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2_approx(x[half * 64 + 2 * k] - msub);
-          const float p1 = ex2_approx(x[half * 64 + 2 * k + 1] - msub);
-          rs += p0 + p1;
+          float e0, e1;
+          f2_unpack(f2_fma(f2_pack(x[half * 64 + 2 * k], x[half * 64 + 2 * k + 1]), sc2, nm2), e0, e1);
+          const float p0 = ex2_approx(e0);
+          const float p1 = ex2_approx(e1);
+          acc[k & 1] = f2_add(acc[k & 1], f2_pack(p0, p1));
           pk[k] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_addr + half * 32, pk);
       }
-      l_sum += rs;
+      {
+        float a0, a1;
+        f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+        l_sum += a0 + a1;
+      }
 
       if (__any_sync(0xffffffffu, rescale_o) && p > 0) {
         // O_h(p-1) is final here: its product was issued before S_h(p).
@@ -458,6 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -469,7 +503,12 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, 
                              const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
                              const CUtensorMap& tm_kr_lo, const PrefillArgs& a, cudaStream_t stream) {
   auto k = bifocal_prefill_kernel<D, kSplit>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, kSplit>::kSmem);
+  // The setmaxnreg split inside the kernel assumes the launch register count.
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, k);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, kSplit>::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Hq / a.nh, a.num_mb, a.B);
   k<<<grid, kThreads, Cfg<D, kSplit>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a);
