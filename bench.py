@@ -165,13 +165,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank timing over all ranks (the only collective the bench
+    makes; no data-path exchange)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank, world, max_ms):
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms * 1e-3)
 
 
 def gen_on_device(shape, seed, dev):
@@ -275,9 +283,9 @@ def run_ours(args):
 
     flop = prefill_flop(P)
     dbytes = decode_bytes(Dc)
-    value = world * flop / (pre_ms_max * 1e-3) / 1e12
+    value = weak_scaling_value(flop, world, pre_ms_max) / 1e12
     attn_tflops = flop / (attn_ms_max * 1e-3) / 1e12
-    dec_gbs = world * dbytes / (dec_ms_max * 1e-3) / 1e9
+    dec_gbs = weak_scaling_value(dbytes, world, dec_ms_max) / 1e9
     dec_gbs_kernel = dbytes / (dec_ms_max * 1e-3) / 1e9
 
     # plain causal RoPE from the same kernels (w0 = L), measured after the timed region
