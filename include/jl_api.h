@@ -169,6 +169,38 @@ int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, i
                       size_t workspace_bytes, int* dev_error, void* stream);
 
 /*
+ * Varlen (continuous-batch) decode: sequence b has its own length
+ * seq_lens[b] (device int32 array, 1 <= seq_lens[b] <= cache_len), hence its
+ * own G_b = max(1, ceil(L_b / w_pretrained)), query position L_b - 1 and band.
+ * The cache is read as it is: a sequence that crosses a multiple of
+ * w_pretrained changes G without any cache rewrite (Jet-Long review, "Method";
+ * gist.science summary, "§2 On-the-Fly Correctie Rotatie").
+ *   max_len: the largest seq_lens value (host side; it sizes the split count).
+ *   Everything else as jl_bifocal_decode; workspace as
+ *   jl_decode_workspace_bytes(B, max_len, Hq, Hkv, head_dim).
+ *   A length outside [1, cache_len] is clamped and flagged in *dev_error (2).
+ * Launches one kernel.
+ */
+int jl_bifocal_decode_varlen(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len,
+                             const int32_t* seq_lens, int max_len, void* o, float* lse, int B, int Hq, int Hkv,
+                             int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale, int mode,
+                             void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
+
+/*
+ * Base RoPE of each sequence's new token and its append to the cache (one
+ * launch).  q_raw [B, Hq, D], k_raw / v_new [B, Hkv, D]: bf16 device, not
+ * rotated.  positions: device int32 [B], the new token's absolute position
+ * p_b (0 <= p_b < cache_len).  Writes q_out [B, Hq, D] = R(p_b) q_raw (the
+ * decode query), k_cache[b, p_b] = R(p_b) k_raw and v_cache[b, p_b] = v_new;
+ * no other cache row is touched.  Angles p_b * theta_t are formed in fp64.
+ * A position out of range skips that sequence and sets *dev_error to 2.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_ALIGNMENT, JL_ERR_CUDA.
+ */
+int jl_rope_append(const void* q_raw, const void* k_raw, const void* v_new, const int32_t* positions, void* q_out,
+                   void* k_cache, void* v_cache, int64_t cache_len, int B, int Hq, int Hkv, int head_dim,
+                   double rope_base, int* dev_error, void* stream);
+
+/*
  * jl_bifocal_decode without a workspace argument, for callers that cannot
  * allocate device memory (e.g. a plugin inside an inference engine whose
  * device memory is wholly owned by the host framework's pool, or a serving

@@ -118,12 +118,25 @@ __global__ void __maxnreg__(168)
   const int lane = threadIdx.x & 31;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int r = args.r;
-  const int L = args.L;
-  const int t_begin = (int)(((int64_t)split * args.ntiles) / args.splits);
-  const int t_end = (int)(((int64_t)(split + 1) * args.ntiles) / args.splits);
-  const int ntile = t_end - t_begin;
-  const int G = (int)args.G;
-  const bool all_local = args.all_local != 0;
+  // This sequence's length and the position algebra that follows from it
+  // (group size, query shift, local band), per CTA so that every sequence of
+  // a varlen batch gets its own G.
+  int L = args.L;
+  if (args.seq_lens != nullptr) {
+    L = args.seq_lens[b];
+    if (L < 1 || (int64_t)L > args.cache_len) {
+      if (threadIdx.x == 0 && args.dev_error) atomicExch(args.dev_error, kDevBadLength);
+      L = L < 1 ? 1 : (int)args.cache_len;
+    }
+  }
+  const int G = (int)group_size(L, args.w_pretrained);
+  const bool all_local = jl::all_local(L, args.w0, G);
+  const int64_t dq = query_remote(L - 1, G, query_shift(args.w0, G, args.qshift)) - (L - 1);
+  const uint32_t g_magic = G < 16 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)G - 1) / (uint64_t)G) : 0u;
+  const int ntiles_b = (L + kDecKeys - 1) / kDecKeys;
+  const int t_begin = (int)(((int64_t)split * ntiles_b) / args.splits);
+  const int t_end = (int)(((int64_t)(split + 1) * ntiles_b) / args.splits);
+  const int ntile = t_end - t_begin;  // may be 0 for short sequences of a varlen batch
   const int local_from = all_local ? 0 : L - args.w0;  // keys j >= local_from are local
 
   if (threadIdx.x == 0) {
@@ -153,7 +166,7 @@ __global__ void __maxnreg__(168)
         turns = -(double)(q64 + (row - 16) - 64);  // -(dk(j0 + 64) - dk(j0))
       } else {
         const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18);
-        turns = (double)(args.dq - (j0 / G - j0));
+        turns = (double)(dq - (j0 / G - j0));
       }
       double sn, cs;
       sincos(turns * args.theta[t], &sn, &cs);
@@ -262,7 +275,7 @@ __global__ void __maxnreg__(168)
   const int q64 = kDecKeys / G, r64 = kDecKeys - q64 * G;
   // floor(x / G) for 0 <= x < G + 16 (one multiply-high; exact there)
   auto div_small = [&](int x) -> int {
-    return G >= 16 ? (x >= G ? 1 : 0) : (int)__umulhi((unsigned)x, args.g_magic);
+    return G >= 16 ? (x >= G ? 1 : 0) : (int)__umulhi((unsigned)x, g_magic);
   };
 
   for (int i = 0; i < ntile; ++i) {

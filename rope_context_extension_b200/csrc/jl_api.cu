@@ -316,28 +316,26 @@ size_t jl_decode_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {
   return decode_layout(B, Hq, Hkv, head_dim, decode_splits_max(B, Hkv)).total;
 }
 
-int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
-                      float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
-                      double rope_base, float softmax_scale, int mode, void* workspace, size_t workspace_bytes,
-                      int* dev_error, void* stream) {
-  const int D = head_dim;
+namespace {
+
+// Shared by the uniform-length and the varlen decode entry points.
+int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len,
+                  const int32_t* seq_lens, int L, void* o, float* lse, int B, int Hq, int Hkv, int D, int w0,
+                  int w_pretrained, double rope_base, float softmax_scale, int mode, void* workspace,
+                  size_t workspace_bytes, int* dev_error, void* stream) {
   int st = common_checks(B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
   if (st != JL_OK) return st;
   if (!q || !k_cache || !v_cache || !o) return JL_ERR_INVALID_ARG;
   if (cache_len < L || cache_len > (int64_t)1 << 31) return JL_ERR_INVALID_ARG;
   if (Hq / Hkv > 8) return JL_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
-      (lse && ((uintptr_t)lse & 3u)))
+      (lse && ((uintptr_t)lse & 3u)) || (seq_lens && ((uintptr_t)seq_lens & 3u)))
     return JL_ERR_ALIGNMENT;
   const int ntiles = (L + 63) / 64;
   const int splits = decode_splits(B, Hkv, ntiles);
   const DecodeLayout lay = decode_layout(B, Hq, Hkv, D, decode_splits_max(B, Hkv));
   if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
-
-  const int64_t G = jl::group_size(L, w_pretrained);
-  const bool all_local = jl::all_local(L, w0, G);
-  const int64_t shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
 
   CUtensorMap tk, tv;
   if (!encode_bf16_4d(&tk, k_cache, D, Hkv, cache_len, B, 64) ||
@@ -354,21 +352,68 @@ int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, i
   a.part_ml = reinterpret_cast<float2*>(ws + lay.ml);
   a.part_o = reinterpret_cast<float*>(ws + lay.o);
   a.dev_error = dev_error;
+  a.seq_lens = seq_lens;
   a.B = B;
   a.L = L;
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.r = Hq / Hkv;
+  a.cache_len = cache_len;
   a.splits = splits;
-  a.ntiles = ntiles;
-  a.w0 = all_local ? (1 << 30) : w0;
-  a.all_local = all_local ? 1 : 0;
-  a.G = G;
-  a.g_magic = G < 16 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)G - 1) / (uint64_t)G) : 0u;
-  a.dq = jl::query_remote(L - 1, G, shift) - (L - 1);
+  a.w0 = w0;
+  a.w_pretrained = w_pretrained;
+  a.qshift = mode & JL_QSHIFT_SELF_EXTEND;
   a.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
   fill_theta(a.theta, D, rope_base);
   if (jl::launch_decode(tk, tv, a, D, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+}  // namespace
+
+int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                      float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
+                      double rope_base, float softmax_scale, int mode, void* workspace, size_t workspace_bytes,
+                      int* dev_error, void* stream) {
+  return decode_launch(q, k_cache, v_cache, cache_len, nullptr, L, o, lse, B, Hq, Hkv, head_dim, w0, w_pretrained,
+                       rope_base, softmax_scale, mode, workspace, workspace_bytes, dev_error, stream);
+}
+
+int jl_bifocal_decode_varlen(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len,
+                             const int32_t* seq_lens, int max_len, void* o, float* lse, int B, int Hq, int Hkv,
+                             int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale, int mode,
+                             void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
+  if (seq_lens == nullptr) return JL_ERR_INVALID_ARG;
+  return decode_launch(q, k_cache, v_cache, cache_len, seq_lens, max_len, o, lse, B, Hq, Hkv, head_dim, w0,
+                       w_pretrained, rope_base, softmax_scale, mode, workspace, workspace_bytes, dev_error, stream);
+}
+
+int jl_rope_append(const void* q_raw, const void* k_raw, const void* v_new, const int32_t* positions, void* q_out,
+                   void* k_cache, void* v_cache, int64_t cache_len, int B, int Hq, int Hkv, int head_dim,
+                   double rope_base, int* dev_error, void* stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || cache_len < 1 || cache_len > (int64_t)1 << 31) return JL_ERR_INVALID_ARG;
+  if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return JL_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return JL_ERR_UNSUPPORTED;
+  if (!q_raw || !k_raw || !v_new || !positions || !q_out || !k_cache || !v_cache) return JL_ERR_INVALID_ARG;
+  if (!aligned16(q_raw) || !aligned16(k_raw) || !aligned16(v_new) || !aligned16(q_out) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || ((uintptr_t)positions & 3u))
+    return JL_ERR_ALIGNMENT;
+  jl::AppendArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q_raw = reinterpret_cast<const __nv_bfloat16*>(q_raw);
+  a.k_raw = reinterpret_cast<const __nv_bfloat16*>(k_raw);
+  a.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+  a.positions = positions;
+  a.q_out = reinterpret_cast<__nv_bfloat16*>(q_out);
+  a.k_cache = reinterpret_cast<__nv_bfloat16*>(k_cache);
+  a.v_cache = reinterpret_cast<__nv_bfloat16*>(v_cache);
+  a.cache_len = cache_len;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.dev_error = dev_error;
+  fill_theta(a.theta, head_dim, rope_base);
+  if (jl::launch_rope_append(a, head_dim, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
 

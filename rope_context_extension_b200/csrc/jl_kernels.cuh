@@ -39,25 +39,42 @@ cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, co
 
 // Split-KV bifocal decode (mma.sync tiles, in-register correction of keys).
 struct DecodeArgs {
-  const __nv_bfloat16* q;  // [B, Hq, D], rotated at position L - 1
+  const __nv_bfloat16* q;  // [B, Hq, D], rotated at position L_b - 1
   __nv_bfloat16* o;        // [B, Hq, D]
   float* lse;              // [B, Hq] or null
   float2* part_ml;         // [B, Hkv, splits, r] (running max in log2 units, sum)
   float* part_o;           // [B, Hkv, splits, r, D]
   int* counters;           // [B, Hkv], zero between calls
   int* dev_error;
-  int B, L, Hq, Hkv, r;
-  int splits, ntiles;      // 64-key tiles in [0, L)
-  int w0, all_local;
-  int64_t G;
-  uint32_t g_magic;        // ceil(2^32 / G) for G < 16 (floor(x / G) = umulhi(x, g_magic), x < 32)
-  int64_t dq;              // p_q(L - 1) - (L - 1)
+  const int* seq_lens;     // [B] per-sequence L_b (device), or null: every L_b = L
+  int B, L, Hq, Hkv, r;    // L: the common length, or the largest L_b
+  int64_t cache_len;       // rows of the cache (bound on L_b)
+  int splits;              // CTAs per (batch, KV head); each covers a share of its sequence's tiles
+  int w0, w_pretrained, qshift;
   float scale_log2;
   double theta[kMaxHalfDim];
 };
+// dev_error value for a sequence length outside [1, cache_len] (varlen decode)
+constexpr int kDevBadLength = 2;
 cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecodeArgs& a, int D,
                           cudaStream_t stream);
 // Resident decode CTAs per SM (occupancy of the D = 128 kernel, cached).
 int decode_ctas_per_sm();
+
+// Base RoPE of one new token per sequence and its append to the KV cache.
+struct AppendArgs {
+  const __nv_bfloat16* q_raw;  // [B, Hq, D] unrotated
+  const __nv_bfloat16* k_raw;  // [B, Hkv, D] unrotated
+  const __nv_bfloat16* v_new;  // [B, Hkv, D]
+  const int* positions;        // [B] absolute position of the new token (device)
+  __nv_bfloat16* q_out;        // [B, Hq, D] rotated at its position
+  __nv_bfloat16* k_cache;      // [B, cache_len, Hkv, D]
+  __nv_bfloat16* v_cache;
+  int64_t cache_len;
+  int B, Hq, Hkv;
+  int* dev_error;
+  double theta[kMaxHalfDim];
+};
+cudaError_t launch_rope_append(const AppendArgs& a, int D, cudaStream_t stream);
 
 }  // namespace jl

@@ -17,7 +17,7 @@ __all__ = [
     "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JL_REMOTE_SPLIT", "JetLongError", "lib", "library_path",
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
-    "jl_bifocal_decode_noalloc", "EXPORTED_SYMBOLS",
+    "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "EXPORTED_SYMBOLS",
 ]
 
 JL_QSHIFT_NONE = 0
@@ -26,7 +26,7 @@ JL_REMOTE_SPLIT = 2  # OR into mode: fp16 hi + lo remote operands in prefill (tw
 EXPORTED_SYMBOLS = (
     "jl_status_string", "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes",
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
-    "jl_prefill_attention", "jl_bifocal_decode_noalloc",
+    "jl_prefill_attention", "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -74,6 +74,11 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_decode_noalloc.argtypes = [c_p, c_p, c_p, c_i64, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d,
                                             c_f, c_i, c_p, c_p]
     L.jl_bifocal_decode_noalloc.restype = c_i
+    L.jl_bifocal_decode_varlen.argtypes = [c_p, c_p, c_p, c_i64, c_p, c_i, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i,
+                                           c_d, c_f, c_i, c_p, c_sz, c_p, c_p]
+    L.jl_bifocal_decode_varlen.restype = c_i
+    L.jl_rope_append.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i, c_i, c_d, c_p, c_p]
+    L.jl_rope_append.restype = c_i
     _lib = L
     return L
 
@@ -226,3 +231,46 @@ def jl_bifocal_decode_noalloc(q, k_cache, v_cache, o, lse, *, L: int, w0: int, w
                                          int(L), Hq, Hkv, D, int(w0), int(w_pretrained), float(rope_base),
                                          float(softmax_scale), int(mode), _ptr(dev_error), _stream(stream))
     _check(st, "jl_bifocal_decode_noalloc")
+
+
+def jl_bifocal_decode_varlen(q, k_cache, v_cache, o, lse, seq_lens, *, max_len: int, w0: int, w_pretrained: int,
+                             rope_base: float, softmax_scale: float = 0.0, mode: int = JL_QSHIFT_SELF_EXTEND,
+                             workspace=None, dev_error=None, stream=None):
+    """Varlen decode: seq_lens is an int32 CUDA tensor [B] of per-sequence lengths
+    (the new token of sequence b sits at seq_lens[b] - 1); max_len >= every length."""
+    import torch
+    B, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    _check_tensor(q, "q", torch.bfloat16)
+    _check_tensor(k_cache, "k_cache", torch.bfloat16)
+    _check_tensor(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
+    _check_tensor(o, "o", torch.bfloat16, (B, Hq, D))
+    _check_tensor(seq_lens, "seq_lens", torch.int32, (B,))
+    if lse is not None:
+        _check_tensor(lse, "lse", torch.float32, (B, Hq))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().jl_bifocal_decode_varlen(_ptr(q), _ptr(k_cache), _ptr(v_cache), Lmax, _ptr(seq_lens), int(max_len),
+                                        _ptr(o), _ptr(lse), B, Hq, Hkv, D, int(w0), int(w_pretrained),
+                                        float(rope_base), float(softmax_scale), int(mode), _ptr(workspace),
+                                        ws_bytes, _ptr(dev_error), _stream(stream))
+    _check(st, "jl_bifocal_decode_varlen")
+
+
+def jl_rope_append(q_raw, k_raw, v_new, positions, q_out, k_cache, v_cache, *, rope_base: float, dev_error=None,
+                   stream=None):
+    """Rotate each sequence's new token at positions[b] (int32 CUDA [B]) and append
+    k / v to cache row positions[b]; q_out receives the rotated query."""
+    import torch
+    B, Hq, D = q_raw.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    _check_tensor(q_raw, "q_raw", torch.bfloat16)
+    _check_tensor(k_raw, "k_raw", torch.bfloat16, (B, Hkv, D))
+    _check_tensor(v_new, "v_new", torch.bfloat16, (B, Hkv, D))
+    _check_tensor(positions, "positions", torch.int32, (B,))
+    _check_tensor(q_out, "q_out", torch.bfloat16, (B, Hq, D))
+    _check_tensor(k_cache, "k_cache", torch.bfloat16)
+    _check_tensor(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
+    st = lib().jl_rope_append(_ptr(q_raw), _ptr(k_raw), _ptr(v_new), _ptr(positions), _ptr(q_out), _ptr(k_cache),
+                              _ptr(v_cache), Lmax, B, Hq, Hkv, D, float(rope_base), _ptr(dev_error),
+                              _stream(stream))
+    _check(st, "jl_rope_append")
