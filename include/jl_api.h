@@ -142,6 +142,36 @@ int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, f
                          const void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
 
 /*
+ * Scratch bytes jl_bifocal_prefill_chunk needs: fp16 corrected rows of the
+ * chunk's queries [B, chunk_len, Hq, D] and of the keys [B, q_offset +
+ * chunk_len, Hkv, D]; twice this with JL_REMOTE_SPLIT.  0 on bad arguments.
+ */
+size_t jl_prefill_chunk_workspace_bytes(int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim);
+
+/*
+ * Chunked prefill against an existing cache: the chunk's queries sit at
+ * positions q_offset .. q_offset + chunk_len - 1 and attend (causally) to
+ * cache keys 0 .. q_offset + chunk_len - 1; G comes from the total length
+ * q_offset + chunk_len (the current length, Jet-Long review "Method").  With
+ * q_offset = 0 and chunk_len = L this is jl_bifocal_prefill on a cache.
+ *   q [B, chunk_len, Hq, D]: bf16 device, rotated at its absolute positions.
+ *   k_cache / v_cache [B, cache_len, Hkv, D]: bf16 device, already holding the
+ *   chunk's own keys and values; read only.  q_offset + chunk_len <= cache_len.
+ *   o [B, chunk_len, Hq, D] bf16; lse [B, Hq, chunk_len] fp32 or NULL.
+ *   workspace: jl_prefill_chunk_workspace_bytes(...) bytes (x2 with
+ *   JL_REMOTE_SPLIT).  Everything else as jl_bifocal_prefill.
+ * Note: a cache built by earlier decode steps is not equivalent to re-running
+ * prefill over the whole sequence (the keys were rotated once, at their base
+ * positions, either way; the hidden states are not recomputed).
+ * Launches: two correction kernels (skipped when every pair is local) and the
+ * fused attention kernel.
+ */
+int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                             float* lse, int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim, int w0,
+                             int w_pretrained, double rope_base, float softmax_scale, int mode, void* workspace,
+                             size_t workspace_bytes, int* dev_error, void* stream);
+
+/*
  * Scratch bytes jl_bifocal_decode needs on this device (split partials and one
  * ticket counter per (batch, KV head)).  0 on bad arguments.
  */

@@ -168,21 +168,138 @@ size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {
   return round_up((size_t)B * L * Hq * head_dim * 2) + round_up((size_t)B * L * Hkv * head_dim * 2);
 }
 
+size_t jl_prefill_chunk_workspace_bytes(int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim) {
+  if (B < 1 || q_offset < 0 || chunk_len < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
+  return round_up((size_t)B * chunk_len * Hq * head_dim * 2) +
+         round_up((size_t)B * ((size_t)q_offset + chunk_len) * Hkv * head_dim * 2);
+}
+
 namespace {
 
-// Shared argument checks of the prefill entry points.
-int prefill_checks(const void* q, const void* k, const void* v, int B, int L, int Hq, int Hkv, int D, int w0,
-                   int w_pretrained, double rope_base, int mode) {
-  int st = common_checks(B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+// One prefill problem: query rows [q_off, q_off + Lq) of every sequence
+// against keys [0, q_off + Lq); Q / O / LSE hold Lq rows, K / V hold k_rows
+// rows (>= q_off + Lq).  G comes from the total length q_off + Lq.
+struct PrefillProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  int B, q_off, Lq, k_rows, Hq, Hkv, D;
+  int Lk() const { return q_off + Lq; }
+  size_t base_ws() const { return jl_prefill_chunk_workspace_bytes(B, q_off, Lq, Hq, Hkv, D); }
+};
+
+__half* q_rem_ptr(void* ws) { return reinterpret_cast<__half*>(ws); }
+__half* k_rem_ptr(void* ws, const PrefillProblem& pp) {
+  return reinterpret_cast<__half*>(reinterpret_cast<char*>(ws) + round_up((size_t)pp.B * pp.Lq * pp.Hq * pp.D * 2));
+}
+
+int problem_checks(const PrefillProblem& pp, int w0, int w_pretrained, double rope_base, int mode) {
+  int st = common_checks(pp.B, pp.Lk(), pp.Hq, pp.Hkv, pp.D, w0, w_pretrained, rope_base, mode);
   if (st != JL_OK) return st;
-  if (!q || !k || !v) return JL_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return JL_ERR_ALIGNMENT;
+  if (pp.q_off < 0 || pp.Lq < 1 || pp.k_rows < pp.Lk()) return JL_ERR_INVALID_ARG;
+  if (!pp.q || !pp.k || !pp.v) return JL_ERR_INVALID_ARG;
+  if (!aligned16(pp.q) || !aligned16(pp.k) || !aligned16(pp.v)) return JL_ERR_ALIGNMENT;
   return JL_OK;
 }
 
-__half* q_rem_ptr(void* ws) { return reinterpret_cast<__half*>(ws); }
-__half* k_rem_ptr(void* ws, int B, int L, int Hq, int D) {
-  return reinterpret_cast<__half*>(reinterpret_cast<char*>(ws) + round_up((size_t)B * L * Hq * D * 2));
+int workspace_checks(const PrefillProblem& pp, int w0, int w_pretrained, int mode, const void* workspace,
+                     size_t workspace_bytes) {
+  const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
+  if (jl::all_local(pp.Lk(), w0, G)) return JL_OK;
+  const size_t need = ((mode & JL_REMOTE_SPLIT) ? 2 : 1) * pp.base_ws();
+  if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
+  return JL_OK;
+}
+
+int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double rope_base, int mode,
+                      void* workspace, cudaStream_t s) {
+  const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
+  if (jl::all_local(pp.Lk(), w0, G)) return JL_OK;  // nothing to correct
+  const bool split = (mode & JL_REMOTE_SPLIT) != 0;
+  char* lo_base = reinterpret_cast<char*>(workspace) + pp.base_ws();  // split: Q_lo then K_lo
+  RotateArgs ra;
+  std::memset(&ra, 0, sizeof(ra));
+  fill_theta(ra.theta, pp.D, rope_base);
+  ra.G = G;
+  ra.shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
+  ra.B = pp.B;
+  // queries that have a remote key: positions q_off + r >= w0
+  ra.x = reinterpret_cast<const __nv_bfloat16*>(pp.q);
+  ra.y = q_rem_ptr(workspace);
+  ra.y_lo = split ? q_rem_ptr(lo_base) : nullptr;
+  ra.x_rows = ra.y_rows = pp.Lq;
+  ra.H = pp.Hq;
+  ra.pos_off = pp.q_off;
+  ra.row_begin = std::max(0, w0 - pp.q_off);
+  ra.row_end = pp.Lq;
+  ra.is_query = 1;
+  if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
+  // keys that have a remote query: j <= q_off + Lq - 1 - w0
+  ra.x = reinterpret_cast<const __nv_bfloat16*>(pp.k);
+  ra.y = k_rem_ptr(workspace, pp);
+  ra.y_lo = split ? k_rem_ptr(lo_base, pp) : nullptr;
+  ra.x_rows = pp.k_rows;
+  ra.y_rows = pp.Lk();
+  ra.H = pp.Hkv;
+  ra.pos_off = 0;
+  ra.row_begin = 0;
+  ra.row_end = pp.Lk() - w0;
+  ra.is_query = 0;
+  if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int attention_launch(const PrefillProblem& pp, void* o, float* lse, int w0, int w_pretrained, float softmax_scale,
+                     int mode, const void* workspace, int* dev_error, cudaStream_t stream) {
+  const int D = pp.D;
+  const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
+  const bool all_local = jl::all_local(pp.Lk(), w0, G);
+  const bool split = !all_local && (mode & JL_REMOTE_SPLIT) != 0;
+  CUtensorMap tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo;
+  if (!encode_bf16_4d(&tq, pp.q, D, pp.Hq, pp.Lq, pp.B, 128) ||
+      !encode_bf16_4d(&tk, pp.k, D, pp.Hkv, pp.k_rows, pp.B, 128) ||
+      !encode_bf16_4d(&tv, pp.v, D, pp.Hkv, pp.k_rows, pp.B, 128))
+    return JL_ERR_CUDA;
+  if (!all_local) {
+    void* ws = const_cast<void*>(workspace);
+    if (!encode_f16_4d(&tqr, q_rem_ptr(ws), D, pp.Hq, pp.Lq, pp.B, 128) ||
+        !encode_f16_4d(&tkr, k_rem_ptr(ws, pp), D, pp.Hkv, pp.Lk(), pp.B, 128))
+      return JL_ERR_CUDA;
+  } else {
+    tqr = tq;
+    tkr = tk;
+  }
+  if (split) {
+    void* lo = reinterpret_cast<char*>(const_cast<void*>(workspace)) + pp.base_ws();
+    if (!encode_f16_4d(&tqr_lo, q_rem_ptr(lo), D, pp.Hq, pp.Lq, pp.B, 128) ||
+        !encode_f16_4d(&tkr_lo, k_rem_ptr(lo, pp), D, pp.Hkv, pp.Lk(), pp.B, 128))
+      return JL_ERR_CUDA;
+  } else {
+    tqr_lo = tqr;
+    tkr_lo = tkr;
+  }
+  const int r = pp.Hq / pp.Hkv;
+  PrefillArgs pa;
+  std::memset(&pa, 0, sizeof(pa));
+  pa.o = reinterpret_cast<__nv_bfloat16*>(o);
+  pa.lse = lse;
+  pa.dev_error = dev_error;
+  pa.B = pp.B;
+  pa.Hq = pp.Hq;
+  pa.Hkv = pp.Hkv;
+  pa.r = r;
+  pa.q_off = pp.q_off;
+  pa.Lq = pp.Lq;
+  pa.Lk = pp.Lk();
+  pa.nh = (!split && r % 2 == 0) ? 2 : 1;
+  pa.num_mb = (pp.Lq + 127) / 128;
+  pa.all_local = all_local ? 1 : 0;
+  pa.w0 = all_local ? (1 << 30) : w0;
+  pa.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
+  if (jl::launch_prefill(tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo, pa, D, split, stream) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
 }
 
 }  // namespace
@@ -190,125 +307,61 @@ __half* k_rem_ptr(void* ws, int B, int L, int Hq, int D) {
 int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, int Hkv, int head_dim, int w0,
                           int w_pretrained, double rope_base, int mode, void* workspace, size_t workspace_bytes,
                           void* stream) {
-  const int D = head_dim;
-  int st = prefill_checks(q, k, k, B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+  const PrefillProblem pp{q, k, k, B, 0, L, L, Hq, Hkv, head_dim};
+  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
+  if (st == JL_OK) st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
   if (st != JL_OK) return st;
-  const int64_t G = jl::group_size(L, w_pretrained);
-  if (jl::all_local(L, w0, G)) return JL_OK;  // nothing to correct
-  const bool split = (mode & JL_REMOTE_SPLIT) != 0;
-  const size_t base_bytes = jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
-  if (!workspace || workspace_bytes < (split ? 2 : 1) * base_bytes) return JL_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  char* lo_base = reinterpret_cast<char*>(workspace) + base_bytes;  // split: Q_lo then K_lo
-  RotateArgs ra;
-  std::memset(&ra, 0, sizeof(ra));
-  fill_theta(ra.theta, D, rope_base);
-  ra.G = G;
-  ra.shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
-  ra.B = B;
-  ra.L = L;
-  // queries that have a remote key: i >= w0
-  ra.x = reinterpret_cast<const __nv_bfloat16*>(q);
-  ra.y = q_rem_ptr(workspace);
-  ra.y_lo = split ? q_rem_ptr(lo_base) : nullptr;
-  ra.H = Hq;
-  ra.row_begin = w0;
-  ra.row_end = L;
-  ra.is_query = 1;
-  if (jl::launch_rotate_rows(ra, D, s) != cudaSuccess) return JL_ERR_CUDA;
-  // keys that have a remote query: j <= L - 1 - w0
-  ra.x = reinterpret_cast<const __nv_bfloat16*>(k);
-  ra.y = k_rem_ptr(workspace, B, L, Hq, D);
-  ra.y_lo = split ? k_rem_ptr(lo_base, B, L, Hq, D) : nullptr;
-  ra.H = Hkv;
-  ra.row_begin = 0;
-  ra.row_end = L - w0;
-  ra.is_query = 0;
-  if (jl::launch_rotate_rows(ra, D, s) != cudaSuccess) return JL_ERR_CUDA;
-  return JL_OK;
+  return correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
                          int Hkv, int head_dim, int w0, int w_pretrained, float softmax_scale, int mode,
                          const void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
-  const int D = head_dim;
-  int st = prefill_checks(q, k, v, B, L, Hq, Hkv, D, w0, w_pretrained, 10000.0, mode);
+  const PrefillProblem pp{q, k, v, B, 0, L, L, Hq, Hkv, head_dim};
+  int st = problem_checks(pp, w0, w_pretrained, 10000.0, mode);
   if (st != JL_OK) return st;
   if (!o) return JL_ERR_INVALID_ARG;
   if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
-  const int64_t G = jl::group_size(L, w_pretrained);
-  const bool all_local = jl::all_local(L, w0, G);
-  const bool split = !all_local && (mode & JL_REMOTE_SPLIT) != 0;
-  const size_t base_bytes = jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
-  if (!all_local) {
-    if (!workspace || workspace_bytes < (split ? 2 : 1) * base_bytes) return JL_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
-  }
-  CUtensorMap tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo;
-  if (!encode_bf16_4d(&tq, q, D, Hq, L, B, 128) || !encode_bf16_4d(&tk, k, D, Hkv, L, B, 128) ||
-      !encode_bf16_4d(&tv, v, D, Hkv, L, B, 128))
-    return JL_ERR_CUDA;
-  if (!all_local) {
-    void* ws = const_cast<void*>(workspace);
-    if (!encode_f16_4d(&tqr, q_rem_ptr(ws), D, Hq, L, B, 128) ||
-        !encode_f16_4d(&tkr, k_rem_ptr(ws, B, L, Hq, D), D, Hkv, L, B, 128))
-      return JL_ERR_CUDA;
-  } else {
-    tqr = tq;
-    tkr = tk;
-  }
-  if (split) {
-    void* lo = reinterpret_cast<char*>(const_cast<void*>(workspace)) + base_bytes;
-    if (!encode_f16_4d(&tqr_lo, q_rem_ptr(lo), D, Hq, L, B, 128) ||
-        !encode_f16_4d(&tkr_lo, k_rem_ptr(lo, B, L, Hq, D), D, Hkv, L, B, 128))
-      return JL_ERR_CUDA;
-  } else {
-    tqr_lo = tqr;
-    tkr_lo = tkr;
-  }
-  const int r = Hq / Hkv;
-  PrefillArgs pa;
-  std::memset(&pa, 0, sizeof(pa));
-  pa.o = reinterpret_cast<__nv_bfloat16*>(o);
-  pa.lse = lse;
-  pa.dev_error = dev_error;
-  pa.B = B;
-  pa.L = L;
-  pa.Hq = Hq;
-  pa.Hkv = Hkv;
-  pa.r = r;
-  pa.nh = (!split && r % 2 == 0) ? 2 : 1;
-  pa.num_mb = (L + 127) / 128;
-  pa.all_local = all_local ? 1 : 0;
-  pa.w0 = all_local ? (1 << 30) : w0;
-  pa.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
-  if (jl::launch_prefill(tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo, pa, D, split,
-                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return JL_ERR_CUDA;
-  return JL_OK;
+  st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
+  if (st != JL_OK) return st;
+  return attention_launch(pp, o, lse, w0, w_pretrained, softmax_scale, mode, workspace, dev_error,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 int jl_bifocal_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
                        int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,
                        int mode, void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
   // Validate everything before the first launch.
-  const int D = head_dim;
-  int st = prefill_checks(q, k, v, B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+  const PrefillProblem pp{q, k, v, B, 0, L, L, Hq, Hkv, head_dim};
+  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
   if (st != JL_OK) return st;
   if (!o) return JL_ERR_INVALID_ARG;
   if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
-  const int64_t G = jl::group_size(L, w_pretrained);
-  if (!jl::all_local(L, w0, G)) {
-    const size_t need = ((mode & JL_REMOTE_SPLIT) ? 2 : 1) * jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
-    if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
-  }
-  st = jl_prefill_correction(q, k, B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode, workspace,
-                             workspace_bytes, stream);
+  st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
   if (st != JL_OK) return st;
-  return jl_prefill_attention(q, k, v, o, lse, B, L, Hq, Hkv, D, w0, w_pretrained, softmax_scale, mode, workspace,
-                              workspace_bytes, dev_error, stream);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s);
+  if (st != JL_OK) return st;
+  return attention_launch(pp, o, lse, w0, w_pretrained, softmax_scale, mode, workspace, dev_error, s);
+}
+
+int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                             float* lse, int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim, int w0,
+                             int w_pretrained, double rope_base, float softmax_scale, int mode, void* workspace,
+                             size_t workspace_bytes, int* dev_error, void* stream) {
+  if (cache_len < 1 || cache_len > ((int64_t)1 << 30)) return JL_ERR_INVALID_ARG;
+  if (q_offset < 0 || chunk_len < 1 || (int64_t)q_offset + chunk_len > cache_len) return JL_ERR_INVALID_ARG;
+  const PrefillProblem pp{q, k_cache, v_cache, B, q_offset, chunk_len, (int)cache_len, Hq, Hkv, head_dim};
+  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
+  if (st != JL_OK) return st;
+  if (!o) return JL_ERR_INVALID_ARG;
+  if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
+  st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
+  if (st != JL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s);
+  if (st != JL_OK) return st;
+  return attention_launch(pp, o, lse, w0, w_pretrained, softmax_scale, mode, workspace, dev_error, s);
 }
 
 size_t jl_decode_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {

@@ -7,12 +7,14 @@ namespace jl {
 
 constexpr int kMaxHalfDim = 64;  // head_dim <= 128
 
-// Correction rotation of rows [row_begin, row_end) of a [B, L, H, D] bf16 tensor.
+// Correction rotation of rows [row_begin, row_end) of x [B, x_rows, H, D] (bf16)
+// into y / y_lo [B, y_rows, H, D] (fp16); row r sits at position r + pos_off.
 struct RotateArgs {
   const __nv_bfloat16* x;
   __half* y;     // fp16 output
   __half* y_lo;  // optional fp16 residual (y + y_lo carries about 22 bits), or null
-  int B, L, H;
+  int B, x_rows, y_rows, H;
+  int pos_off;
   int row_begin, row_end;
   int is_query;      // 1: rotate by p_q(i) - i, 0: by f(j) - j
   int64_t G, shift;  // group size and query shift
@@ -22,12 +24,15 @@ cudaError_t launch_rotate_rows(const RotateArgs& args, int D, cudaStream_t strea
 
 // Fused bifocal prefill (tcgen05 + TMEM + TMA).
 struct PrefillArgs {
-  __nv_bfloat16* o;  // [B, L, Hq, D]
-  float* lse;        // [B, Hq, L] or null
+  __nv_bfloat16* o;  // [B, Lq, Hq, D]
+  float* lse;        // [B, Hq, Lq] or null
   int* dev_error;    // device int or null
-  int B, L, Hq, Hkv, r;
+  int B, Hq, Hkv, r;
+  int q_off;         // position of query row 0 (0 for a whole-sequence prefill)
+  int Lq;            // query rows (this chunk)
+  int Lk;            // keys: q_off + Lq
   int nh;            // query heads per CTA (1 or 2, same KV head)
-  int num_mb;        // ceil(L / 128)
+  int num_mb;        // ceil(Lq / 128)
   int w0;            // band width; huge when every pair is local
   int all_local;
   float scale_log2;  // softmax scale * log2(e)

@@ -80,27 +80,39 @@ enum {
 };
 static_assert(kNumBars * 8 <= 192, "barrier block overflow");
 
-// Pass schedule of one query block mb: n_loc local passes on key blocks
-// mb, mb-1, ... then n_rem remote passes on key blocks mb - a_min, ..., 0.
+// Pass schedule of one query block whose first query position is `off`
+// (query rows off .. off + 127; keys in 128-key blocks nb).  Block nb spans
+// i - j in [off - 128 nb - 127, off - 128 nb + 127].  Local passes run on the
+// key blocks nb_max, nb_max - 1, ... that hold a pair with 0 <= i - j < w0;
+// remote passes on nb_rem_max, ..., 0 (the blocks with a pair i - j >= w0).
 struct Sched {
-  int n_loc, n_rem, a_min;
+  int n_loc, n_rem, nb_max, nb_rem_max;
 };
 
-__device__ __forceinline__ Sched make_sched(int mb, int w0, bool all_local) {
+__device__ __forceinline__ int floor_div128(int x) { return x >= 0 ? x / 128 : -((127 - x) / 128); }
+
+__device__ __forceinline__ Sched make_sched(int off, int w0, bool all_local) {
   Sched s;
+  s.nb_max = (off + 127) / 128;  // last block holding a causal key
   if (all_local) {
-    s.n_loc = mb + 1;
+    s.n_loc = s.nb_max + 1;
     s.n_rem = 0;
-    s.a_min = mb + 1;
+    s.nb_rem_max = -1;
     return s;
   }
-  // block distance a = mb - nb spans i - j in [128a - 127, 128a + 127]
-  // local pairs exist iff w0 > 0 and 128a - 127 < w0
-  s.n_loc = (w0 > 0) ? min(mb, (w0 + 126) / 128) + 1 : 0;
-  // remote pairs exist iff 128a + 127 >= w0
-  s.a_min = w0 / 128;
-  s.n_rem = max(0, mb - s.a_min + 1);
+  if (w0 > 0) {
+    const int nb_loc_min = max(0, floor_div128(off - 127 - w0) + 1);  // 128 nb > off - 127 - w0
+    s.n_loc = max(0, s.nb_max - nb_loc_min + 1);
+  } else {
+    s.n_loc = 0;
+  }
+  s.nb_rem_max = floor_div128(off + 127 - w0);  // 128 nb <= off + 127 - w0
+  s.n_rem = max(0, s.nb_rem_max + 1);
   return s;
+}
+
+__device__ __forceinline__ int pass_block(const Sched& s, int p) {
+  return p < s.n_loc ? s.nb_max - p : s.nb_rem_max - (p - s.n_loc);
 }
 
 __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
@@ -167,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
 
-  const Sched sc = make_sched(mb, args.w0, args.all_local != 0);
+  const int off = args.q_off + mb * kBM;  // position of this block's first query
+  const Sched sc = make_sched(off, args.w0, args.all_local != 0);
   const int npass = sc.n_loc + sc.n_rem;
   const bool q_switch = sc.n_loc > 0 && sc.n_rem > 0;
   const int w0 = args.w0;
@@ -220,8 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sv = p % C::kVStages;
         const uint32_t phv = (uint32_t)(p / C::kVStages) & 1u;
         const bool remote = p >= sc.n_loc;
-        const int a = remote ? sc.a_min + (p - sc.n_loc) : p;
-        const int nb = mb - a;
+        const int nb = pass_block(sc, p);
         if (q_switch && p == sc.n_loc) {
           if (!(ok = mbar_wait(bar(kQEmpty), 0, abort_flag, args.dev_error))) break;
           load_q(true);
@@ -366,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const bool remote = p >= sc.n_loc;
-      const int a = remote ? sc.a_min + (p - sc.n_loc) : p;
+      const int dd0 = off - 128 * pass_block(sc, p);  // i - j at row 0, column 0
 
       uint32_t sr[4][32];
 #pragma unroll
@@ -380,9 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]);
 
-      const bool need_mask = remote ? (128 * a - 127 < w0) : (a == 0 || 128 * a + 127 >= w0);
+      const bool need_mask = remote ? (dd0 - 127 < w0) : (dd0 - 127 < 0 || dd0 + 127 >= w0);
       if (need_mask) {
-        const int dd = 128 * a + row;  // i - j = dd - col
+        const int dd = dd0 + row;  // i - j = dd - col
 #pragma unroll
         for (int col = 0; col < 128; ++col) {
           const int rel = dd - col;
@@ -465,9 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      const int i = mb * kBM + row;
+      const int i = mb * kBM + row;  // row of this chunk's Q / O / LSE
       const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      __nv_bfloat16* orow = args.o + (((size_t)b * args.L + i) * args.Hq + hq) * D;
+      __nv_bfloat16* orow = args.o + (((size_t)b * args.Lq + i) * args.Hq + hq) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -477,15 +489,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 16; ++k)
           w[k] = pack_bf16x2(__uint_as_float(ov[2 * k]) * inv, __uint_as_float(ov[2 * k + 1]) * inv);
-        if (i < args.L) {
+        if (i < args.Lq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
-      if (args.lse != nullptr && i < args.L) {
+      if (args.lse != nullptr && i < args.Lq) {
         const float m = (m_used == -INFINITY) ? 0.f : m_used;
-        args.lse[((size_t)b * args.Hq + hq) * args.L + i] = (m + __log2f(l_sum)) * 0.69314718055994531f;
+        args.lse[((size_t)b * args.Hq + hq) * args.Lq + i] = (m + __log2f(l_sum)) * 0.69314718055994531f;
       }
     }
   }

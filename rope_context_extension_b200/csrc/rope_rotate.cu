@@ -37,8 +37,9 @@ __global__ void __launch_bounds__(kRotThreads)
     const int64_t i = row0 + r;
     float2 v = make_float2(1.f, 0.f);
     if (i < args.row_end) {
-      const int64_t target = args.is_query ? query_remote(i, args.G, args.shift) : key_remote(i, args.G);
-      const double ang = (double)(target - i) * args.theta[t];
+      const int64_t pos = i + args.pos_off;
+      const int64_t target = args.is_query ? query_remote(pos, args.G, args.shift) : key_remote(pos, args.G);
+      const double ang = (double)(target - pos) * args.theta[t];
       double s, c;
       sincos(ang, &s, &c);
       v = make_float2((float)c, (float)s);
@@ -55,9 +56,10 @@ __global__ void __launch_bounds__(kRotThreads)
     const int r = w / (kChunks * args.H);
     const int64_t i = row0 + r;
     if (i >= args.row_end) continue;
-    const size_t base = (((size_t)b * args.L + i) * args.H + h) * D;
-    const uint4 lo = *reinterpret_cast<const uint4*>(args.x + base + ch * 8);
-    const uint4 hi = *reinterpret_cast<const uint4*>(args.x + base + H2 + ch * 8);
+    const size_t xbase = (((size_t)b * args.x_rows + i) * args.H + h) * D;
+    const size_t base = (((size_t)b * args.y_rows + i) * args.H + h) * D;
+    const uint4 lo = *reinterpret_cast<const uint4*>(args.x + xbase + ch * 8);
+    const uint4 hi = *reinterpret_cast<const uint4*>(args.x + xbase + H2 + ch * 8);
     const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w};
     const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w};
     float rx[8], ry[8];

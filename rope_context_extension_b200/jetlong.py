@@ -17,7 +17,8 @@ __all__ = [
     "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JL_REMOTE_SPLIT", "JetLongError", "lib", "library_path",
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
-    "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "EXPORTED_SYMBOLS",
+    "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
+    "jl_bifocal_prefill_chunk", "EXPORTED_SYMBOLS",
 ]
 
 JL_QSHIFT_NONE = 0
@@ -27,6 +28,7 @@ EXPORTED_SYMBOLS = (
     "jl_status_string", "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes",
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
     "jl_prefill_attention", "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append",
+    "jl_prefill_chunk_workspace_bytes", "jl_bifocal_prefill_chunk",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -79,6 +81,11 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_decode_varlen.restype = c_i
     L.jl_rope_append.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i, c_i, c_d, c_p, c_p]
     L.jl_rope_append.restype = c_i
+    L.jl_prefill_chunk_workspace_bytes.argtypes = [c_i, c_i, c_i, c_i, c_i, c_i]
+    L.jl_prefill_chunk_workspace_bytes.restype = c_sz
+    L.jl_bifocal_prefill_chunk.argtypes = [c_p, c_p, c_p, c_i64, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_i,
+                                           c_d, c_f, c_i, c_p, c_sz, c_p, c_p]
+    L.jl_bifocal_prefill_chunk.restype = c_i
     _lib = L
     return L
 
@@ -274,3 +281,29 @@ def jl_rope_append(q_raw, k_raw, v_new, positions, q_out, k_cache, v_cache, *, r
                               _ptr(v_cache), Lmax, B, Hq, Hkv, D, float(rope_base), _ptr(dev_error),
                               _stream(stream))
     _check(st, "jl_rope_append")
+
+
+def jl_prefill_chunk_workspace_bytes(B: int, q_offset: int, chunk_len: int, Hq: int, Hkv: int, head_dim: int) -> int:
+    return int(lib().jl_prefill_chunk_workspace_bytes(B, q_offset, chunk_len, Hq, Hkv, head_dim))
+
+
+def jl_bifocal_prefill_chunk(q, k_cache, v_cache, o, lse, *, q_offset: int, w0: int, w_pretrained: int,
+                             rope_base: float, softmax_scale: float = 0.0, mode: int = JL_QSHIFT_SELF_EXTEND,
+                             workspace=None, dev_error=None, stream=None):
+    """Chunked prefill: q [B, C, Hq, D] at positions q_offset..q_offset+C-1 against
+    cache rows 0..q_offset+C-1 (the cache already holds the chunk's keys)."""
+    import torch
+    B, C, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    _check_tensor(q, "q", torch.bfloat16)
+    _check_tensor(k_cache, "k_cache", torch.bfloat16)
+    _check_tensor(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
+    _check_tensor(o, "o", torch.bfloat16, (B, C, Hq, D))
+    if lse is not None:
+        _check_tensor(lse, "lse", torch.float32, (B, Hq, C))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().jl_bifocal_prefill_chunk(_ptr(q), _ptr(k_cache), _ptr(v_cache), Lmax, _ptr(o), _ptr(lse), B,
+                                        int(q_offset), C, Hq, Hkv, D, int(w0), int(w_pretrained), float(rope_base),
+                                        float(softmax_scale), int(mode), _ptr(workspace), ws_bytes, _ptr(dev_error),
+                                        _stream(stream))
+    _check(st, "jl_bifocal_prefill_chunk")

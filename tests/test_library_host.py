@@ -135,3 +135,23 @@ def test_decode_argument_errors(lib):
 def test_status_strings(lib):
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert lib.jl_status_string(code)
+
+
+def test_prefill_chunk_argument_errors(lib):
+    def chunk(q_offset=100, chunk_len=156, cache_len=256, **kw):
+        a = dict(q=A, k=A, v=A, o=A, lse=None, B=1, Hq=4, Hkv=2, D=128, w0=16, W=64, base=1e4, scale=0.0, mode=1,
+                 ws=A, ws_bytes=1 << 40)
+        a.update(kw)
+        return lib.jl_bifocal_prefill_chunk(a["q"], a["k"], a["v"], cache_len, a["o"], a["lse"], a["B"], q_offset,
+                                            chunk_len, a["Hq"], a["Hkv"], a["D"], a["w0"], a["W"], a["base"],
+                                            a["scale"], a["mode"], a["ws"], a["ws_bytes"], None, None)
+    assert chunk(q_offset=200) == JL_ERR_INVALID_ARG       # chunk runs past the cache
+    assert chunk(q_offset=-1) == JL_ERR_INVALID_ARG
+    assert chunk(chunk_len=0) == JL_ERR_INVALID_ARG
+    assert chunk(D=80) == JL_ERR_UNSUPPORTED
+    assert chunk(k=A + 4) == JL_ERR_ALIGNMENT
+    need = lib.jl_prefill_chunk_workspace_bytes(1, 100, 156, 4, 2, 128)
+    assert need == jl.jl_prefill_chunk_workspace_bytes(1, 100, 156, 4, 2, 128) > 0
+    assert chunk(ws_bytes=need - 1) == JL_ERR_WORKSPACE
+    # a whole-sequence chunk needs what jl_prefill_workspace_bytes reports
+    assert lib.jl_prefill_chunk_workspace_bytes(2, 0, 300, 8, 2, 64) == lib.jl_prefill_workspace_bytes(2, 300, 8, 2, 64)
