@@ -302,6 +302,15 @@ def run_ours(args):
 
     plain_pre_ms = time_calls(lambda: prefill_step(w0=P["L"]), max(2, K // 2))
     plain_dec_ms = time_calls(lambda: decode_step(w0=Dc["L"]), max(2, K // 2))
+    # the pages' unfused three-call inclusion-exclusion formulation, same inputs
+    ie_ms = None
+    if not args.no_ie:
+        ws3 = torch.empty(jl.jl_prefill_ie_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]),
+                          dtype=torch.uint8, device=dev)
+        ie_ms = time_calls(lambda: jl.jl_bifocal_prefill_ie(q, k, v, o, lse, w0=P["w0"], w_pretrained=P["W"],
+                                                            rope_base=P["base"], workspace=ws3, dev_error=err,
+                                                            stream=stream), 2)
+        del ws3
     # split-precision remote products (for inputs with dominant large-norm keys)
     split_pre_ms = None
     if not args.no_split:
@@ -376,6 +385,9 @@ def run_ours(args):
                                     "frac": round(dec_gbs_kernel / peaks["hbm_gbs"], 4),
                                     "traffic": traffic.get("decode", {}).get("bytes_per_launch"),
                                     "peak_source": f"{peak_kind} hbm_gbs"}},
+            "prefill_inclusion_exclusion_3pass": None if ie_ms is None else {
+                "ms": round(ie_ms, 3), "tflops": round(flop / (ie_ms * 1e-3) / 1e12, 2),
+                "fused_speedup": round(ie_ms / pre_ms_max, 3)},
             "prefill_split_precision": None if split_pre_ms is None else {
                 "ms": round(split_pre_ms, 3), "tflops": round(flop / (split_pre_ms * 1e-3) / 1e12, 2)},
             "plain_rope_same_kernels": {
@@ -492,6 +504,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-split", action="store_true", help="skip the split-precision prefill measurement")
+    ap.add_argument("--no-ie", action="store_true", help="skip the three-call inclusion-exclusion measurement")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=4)
     ap.add_argument("--prefill-len", type=int, default=None, help="smaller prefill L (profiling runs only)")

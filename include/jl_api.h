@@ -172,6 +172,30 @@ int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_c
                              size_t workspace_bytes, int* dev_error, void* stream);
 
 /*
+ * Scratch bytes jl_bifocal_prefill_ie needs (for the given mode): corrected
+ * rows for every position, plus three partial outputs and their LSEs.
+ */
+size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim, int mode);
+
+/*
+ * The pages' own prefill formulation, unfused, for comparison with the fused
+ * per-tile kernel (Jet-Long review, "Method"; gist.science summary, "§2
+ * Inclusie-Exclusie Attention Merge"): three attention calls — (A) the window
+ * 0 <= i - j < w0 with base RoPE, (B) every causal pair with remote positions,
+ * (C) the window with remote positions — each writing a bf16 output and an
+ * fp32 LSE, merged as O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C),
+ * W_X = exp(LSE_X - max LSE).  Same arguments and result as jl_bifocal_prefill
+ * (up to the rounding of the partial outputs, which the subtraction
+ * amplifies); workspace: jl_prefill_ie_workspace_bytes(...).  When every pair
+ * is local it runs jl_bifocal_prefill.
+ * Launches: two correction kernels (all rows), three attention kernels, one
+ * merge kernel.
+ */
+int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
+                          int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,
+                          int mode, void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
+
+/*
  * Scratch bytes jl_bifocal_decode needs on this device (split partials and one
  * ticket counter per (batch, KV head)).  0 on bad arguments.
  */

@@ -1,0 +1,59 @@
+// Inclusion-exclusion merge of the three calls of the pages' prefill
+// formulation (Jet-Long review, "Method"):
+//   O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C),  W_X = exp(LSE_X - M),
+//   LSE = M + ln(W_A + W_B - W_C),  M = max(LSE_A, LSE_B, LSE_C),
+// where A is the window with base RoPE, B every causal pair with remote
+// positions and C the window with remote positions; C removes exactly the part
+// of B that A replaces.  The three partial outputs arrive in bf16, as a
+// FlashAttention call returns them, so the subtraction W_B O_B - W_C O_C sees
+// their rounding.  One warp per (sequence, row, head); memory bound.
+#include "jl_kernels.cuh"
+
+namespace jl {
+
+namespace {
+
+template <int D>
+__global__ void __launch_bounds__(256) ie_merge_kernel(const __grid_constant__ MergeArgs a) {
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)a.B * a.L * a.Hq;
+  if (warp_global >= rows) return;
+  const int h = (int)(warp_global % a.Hq);
+  const int64_t bi = warp_global / a.Hq;
+  const int i = (int)(bi % a.L);
+  const int b = (int)(bi / a.L);
+  const size_t lidx = ((size_t)b * a.Hq + h) * a.L + i;
+  const float la = a.lse_x[0][lidx], lb = a.lse_x[1][lidx], lc = a.lse_x[2][lidx];
+  const float M = fmaxf(fmaxf(la, lb), lc);
+  const float wa = la == -INFINITY ? 0.f : expf(la - M);
+  const float wb = lb == -INFINITY ? 0.f : expf(lb - M);
+  const float wc = lc == -INFINITY ? 0.f : expf(lc - M);
+  const float den = wa + wb - wc;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const size_t obase = ((size_t)bi * a.Hq + h) * D;
+  constexpr int kPer = D / 32;  // elements per lane
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int d = lane + 32 * e;
+    const float oa = __bfloat162float(a.o_x[0][obase + d]);
+    const float ob = __bfloat162float(a.o_x[1][obase + d]);
+    const float oc = __bfloat162float(a.o_x[2][obase + d]);
+    a.o[obase + d] = __float2bfloat16_rn((wa * oa + wb * ob - wc * oc) * inv);
+  }
+  if (lane == 0 && a.lse != nullptr) a.lse[lidx] = M + logf(den);
+}
+
+}  // namespace
+
+cudaError_t launch_ie_merge(const MergeArgs& a, int D, cudaStream_t stream) {
+  const int64_t rows = (int64_t)a.B * a.L * a.Hq;
+  const int64_t blocks = (rows * 32 + 255) / 256;
+  if (D == 128)
+    ie_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  else
+    ie_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace jl

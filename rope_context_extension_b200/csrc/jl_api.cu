@@ -213,7 +213,7 @@ int workspace_checks(const PrefillProblem& pp, int w0, int w_pretrained, int mod
 }
 
 int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double rope_base, int mode,
-                      void* workspace, cudaStream_t s) {
+                      void* workspace, cudaStream_t s, bool all_rows = false) {
   const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
   if (jl::all_local(pp.Lk(), w0, G)) return JL_OK;  // nothing to correct
   const bool split = (mode & JL_REMOTE_SPLIT) != 0;
@@ -231,7 +231,7 @@ int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double
   ra.x_rows = ra.y_rows = pp.Lq;
   ra.H = pp.Hq;
   ra.pos_off = pp.q_off;
-  ra.row_begin = std::max(0, w0 - pp.q_off);
+  ra.row_begin = all_rows ? 0 : std::max(0, w0 - pp.q_off);
   ra.row_end = pp.Lq;
   ra.is_query = 1;
   if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
@@ -244,17 +244,17 @@ int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double
   ra.H = pp.Hkv;
   ra.pos_off = 0;
   ra.row_begin = 0;
-  ra.row_end = pp.Lk() - w0;
+  ra.row_end = all_rows ? pp.Lk() : pp.Lk() - w0;
   ra.is_query = 0;
   if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
 
 int attention_launch(const PrefillProblem& pp, void* o, float* lse, int w0, int w_pretrained, float softmax_scale,
-                     int mode, const void* workspace, int* dev_error, cudaStream_t stream) {
+                     int mode, const void* workspace, int* dev_error, cudaStream_t stream, int kind = jl::kBifocal) {
   const int D = pp.D;
   const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
-  const bool all_local = jl::all_local(pp.Lk(), w0, G);
+  const bool all_local = kind == jl::kBifocal && jl::all_local(pp.Lk(), w0, G);
   const bool split = !all_local && (mode & JL_REMOTE_SPLIT) != 0;
   CUtensorMap tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo;
   if (!encode_bf16_4d(&tq, pp.q, D, pp.Hq, pp.Lq, pp.B, 128) ||
@@ -296,6 +296,7 @@ int attention_launch(const PrefillProblem& pp, void* o, float* lse, int w0, int 
   pa.num_mb = (pp.Lq + 127) / 128;
   pa.all_local = all_local ? 1 : 0;
   pa.w0 = all_local ? (1 << 30) : w0;
+  pa.kind = kind;
   pa.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
   if (jl::launch_prefill(tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo, pa, D, split, stream) != cudaSuccess)
     return JL_ERR_CUDA;
@@ -362,6 +363,75 @@ int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_c
   st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s);
   if (st != JL_OK) return st;
   return attention_launch(pp, o, lse, w0, w_pretrained, softmax_scale, mode, workspace, dev_error, s);
+}
+
+namespace {
+
+struct IeLayout {
+  size_t o[3], lse[3], total;
+};
+IeLayout ie_layout(int B, int L, int Hq, int Hkv, int D, int mode) {
+  IeLayout lay;
+  size_t off = ((mode & JL_REMOTE_SPLIT) ? 2 : 1) * jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
+  for (int x = 0; x < 3; ++x) {
+    lay.o[x] = off;
+    off += round_up((size_t)B * L * Hq * D * 2);
+  }
+  for (int x = 0; x < 3; ++x) {
+    lay.lse[x] = off;
+    off += round_up((size_t)B * Hq * L * 4);
+  }
+  lay.total = off;
+  return lay;
+}
+
+}  // namespace
+
+size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim, int mode) {
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
+  return ie_layout(B, L, Hq, Hkv, head_dim, mode).total;
+}
+
+int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
+                          int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,
+                          int mode, void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
+  const PrefillProblem pp{q, k, v, B, 0, L, L, Hq, Hkv, head_dim};
+  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
+  if (st != JL_OK) return st;
+  if (!o) return JL_ERR_INVALID_ARG;
+  if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
+  const int64_t G = jl::group_size(L, w_pretrained);
+  if (jl::all_local(L, w0, G)) {
+    // every pair local: the three calls collapse to plain causal attention
+    return jl_bifocal_prefill(q, k, v, o, lse, B, L, Hq, Hkv, head_dim, w0, w_pretrained, rope_base, softmax_scale,
+                              mode, workspace, workspace_bytes, dev_error, stream);
+  }
+  const IeLayout lay = ie_layout(B, L, Hq, Hkv, head_dim, mode);
+  if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = reinterpret_cast<char*>(workspace);
+  // call B scores every causal pair with corrected rows: correct all rows
+  st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s, /*all_rows=*/true);
+  if (st != JL_OK) return st;
+  const int kinds[3] = {jl::kWindowBase, jl::kCausalRemote, jl::kWindowRemote};
+  jl::MergeArgs ma;
+  std::memset(&ma, 0, sizeof(ma));
+  for (int x = 0; x < 3; ++x) {
+    void* ox = ws + lay.o[x];
+    float* lx = reinterpret_cast<float*>(ws + lay.lse[x]);
+    st = attention_launch(pp, ox, lx, w0, w_pretrained, softmax_scale, mode, workspace, dev_error, s, kinds[x]);
+    if (st != JL_OK) return st;
+    ma.o_x[x] = reinterpret_cast<const __nv_bfloat16*>(ox);
+    ma.lse_x[x] = lx;
+  }
+  ma.o = reinterpret_cast<__nv_bfloat16*>(o);
+  ma.lse = lse;
+  ma.B = B;
+  ma.L = L;
+  ma.Hq = Hq;
+  if (jl::launch_ie_merge(ma, head_dim, s) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
 }
 
 size_t jl_decode_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {

@@ -35,8 +35,10 @@ struct PrefillArgs {
   int num_mb;        // ceil(Lq / 128)
   int w0;            // band width; huge when every pair is local
   int all_local;
+  int kind;          // kBifocal, or one call of the inclusion-exclusion formulation
   float scale_log2;  // softmax scale * log2(e)
 };
+enum : int { kBifocal = 0, kWindowBase = 1, kCausalRemote = 2, kWindowRemote = 3 };
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
                            const CUtensorMap& tm_kr_lo, const PrefillArgs& a, int D, bool split,
@@ -65,6 +67,16 @@ cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, cons
                           cudaStream_t stream);
 // Resident decode CTAs per SM (occupancy of the D = 128 kernel, cached).
 int decode_ctas_per_sm();
+
+// Inclusion-exclusion merge of three partial prefill outputs.
+struct MergeArgs {
+  const __nv_bfloat16* o_x[3];  // O_A, O_B, O_C [B, L, Hq, D]
+  const float* lse_x[3];        // LSE_A, LSE_B, LSE_C [B, Hq, L] (natural log)
+  __nv_bfloat16* o;
+  float* lse;                   // or null
+  int B, L, Hq;
+};
+cudaError_t launch_ie_merge(const MergeArgs& a, int D, cudaStream_t stream);
 
 // Base RoPE of one new token per sequence and its append to the KV cache.
 struct AppendArgs {

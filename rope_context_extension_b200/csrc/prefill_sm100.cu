@@ -87,13 +87,26 @@ static_assert(kNumBars * 8 <= 192, "barrier block overflow");
 // remote passes on nb_rem_max, ..., 0 (the blocks with a pair i - j >= w0).
 struct Sched {
   int n_loc, n_rem, nb_max, nb_rem_max;
+  int kind;
 };
 
 __device__ __forceinline__ int floor_div128(int x) { return x >= 0 ? x / 128 : -((127 - x) / 128); }
 
-__device__ __forceinline__ Sched make_sched(int off, int w0, bool all_local) {
+// kind: kBifocal (local passes, then remote passes: the fused method), or one
+// of the three calls of the inclusion-exclusion formulation (Jet-Long review,
+// "Method"): kWindowBase (A: pairs with 0 <= i - j < w0, base rows),
+// kCausalRemote (B: every causal pair, corrected rows), kWindowRemote (C: the
+// window of A, corrected rows).
+__device__ __forceinline__ Sched make_sched(int off, int w0, bool all_local, int kind) {
   Sched s;
+  s.kind = kind;
   s.nb_max = (off + 127) / 128;  // last block holding a causal key
+  if (kind == kCausalRemote) {
+    s.n_loc = 0;
+    s.nb_rem_max = s.nb_max;
+    s.n_rem = s.nb_max + 1;
+    return s;
+  }
   if (all_local) {
     s.n_loc = s.nb_max + 1;
     s.n_rem = 0;
@@ -107,12 +120,22 @@ __device__ __forceinline__ Sched make_sched(int off, int w0, bool all_local) {
     s.n_loc = 0;
   }
   s.nb_rem_max = floor_div128(off + 127 - w0);  // 128 nb <= off + 127 - w0
-  s.n_rem = max(0, s.nb_rem_max + 1);
+  s.n_rem = kind == kBifocal ? max(0, s.nb_rem_max + 1) : 0;
   return s;
 }
 
 __device__ __forceinline__ int pass_block(const Sched& s, int p) {
   return p < s.n_loc ? s.nb_max - p : s.nb_rem_max - (p - s.n_loc);
+}
+// Does pass p read the corrected (remote-position) Q / K rows?
+__device__ __forceinline__ bool pass_remote_ops(const Sched& s, int p) {
+  return s.kind == kBifocal ? p >= s.n_loc : (s.kind != kWindowBase);
+}
+// Which pairs of the tile pass p keeps: 0 band (0 <= i-j < w0), 1 beyond the
+// band (i-j >= w0), 2 every causal pair (i-j >= 0).
+__device__ __forceinline__ int pass_mask_kind(const Sched& s, int p) {
+  if (s.kind == kCausalRemote) return 2;
+  return p < s.n_loc ? 0 : 1;
 }
 
 __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
@@ -180,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
   const int off = args.q_off + mb * kBM;  // position of this block's first query
-  const Sched sc = make_sched(off, args.w0, args.all_local != 0);
+  const Sched sc = make_sched(off, args.w0, args.all_local != 0, args.kind);
   const int npass = sc.n_loc + sc.n_rem;
   const bool q_switch = sc.n_loc > 0 && sc.n_rem > 0;
   const int w0 = args.w0;
@@ -223,8 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(sbase + C::kQOff + hh * C::kTileBytes + c * kChunkBytes, m, bar(kQFull), c * 64,
                         hq0 + hh, mb * kBM, b);
       };
-      load_q(sc.n_loc == 0);
-      int q_loads = 1;
+      // A query block with no pass (a window call with w0 = 0) loads nothing.
+      if (npass > 0) load_q(pass_remote_ops(sc, 0));
+      int q_loads = npass > 0 ? 1 : 0;
       int k_last = -1, v_last = -1;  // last passes whose K / V copies were issued
       bool ok = true;
       for (int p = 0; p < npass; ++p) {
@@ -232,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (uint32_t)(p / kStages) & 1u;
         const int sv = p % C::kVStages;
         const uint32_t phv = (uint32_t)(p / C::kVStages) & 1u;
-        const bool remote = p >= sc.n_loc;
+        const bool remote = pass_remote_ops(sc, p);
         const int nb = pass_block(sc, p);
         if (q_switch && p == sc.n_loc) {
           if (!(ok = mbar_wait(bar(kQEmpty), 0, abort_flag, args.dev_error))) break;
@@ -259,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // Let every copy already issued land before the CTA can exit.
-        drain_wait(bar(kQFull), (uint32_t)(q_loads - 1) & 1u);
+        if (q_loads > 0) drain_wait(bar(kQFull), (uint32_t)(q_loads - 1) & 1u);
         for (int p = max(0, k_last - kStages + 1); p <= k_last; ++p)
           drain_wait(bar(kKFull + p % kStages), (uint32_t)(p / kStages) & 1u);
         for (int p = max(0, v_last - C::kVStages + 1); p <= v_last; ++p)
@@ -272,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_s_loc = make_idesc_16bit(kBM, kBN, false, false);  // bf16 Q K
       const uint32_t id_s_rem = make_idesc_16bit(kBM, kBN, false, true);   // fp16 Q_rem K_rem
       const uint32_t id_pv = make_idesc_16bit(kBM, D, true, false);        // bf16 P V
-      bool ok = mbar_wait(bar(kQFull), 0, abort_flag, args.dev_error);
+      bool ok = npass == 0 || mbar_wait(bar(kQFull), 0, abort_flag, args.dev_error);
       auto s_col = [&](int h) -> uint32_t { return (uint32_t)(h * 128); };
       auto o_col = [&](int h) -> uint32_t { return (uint32_t)(NH * 128 + h * D); };
 
@@ -286,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t qa = sbase + C::kQOff + h * C::kTileBytes;
         const uint32_t ka = sbase + C::kKOff + s * C::kKSlots * C::kTileBytes;
-        const bool remote = p >= sc.n_loc;
+        const bool remote = pass_remote_ops(sc, p);
         const uint32_t id_s = remote ? id_s_rem : id_s_loc;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -335,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
-      if (ok) {
+      if (ok && npass > 0) {
         if (NH == 2) {
           ok = issue_s(0, 0) && issue_s(1, 0) && issue_pv(0, 0);
           for (int p = 1; p < npass && ok; ++p) {
@@ -377,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const bool remote = p >= sc.n_loc;
+      const int mkind = pass_mask_kind(sc, p);
       const int dd0 = off - 128 * pass_block(sc, p);  // i - j at row 0, column 0
 
       uint32_t sr[4][32];
@@ -392,13 +416,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]);
 
-      const bool need_mask = remote ? (dd0 - 127 < w0) : (dd0 - 127 < 0 || dd0 + 127 >= w0);
+      const bool need_mask = mkind == 1 ? (dd0 - 127 < w0)
+                             : mkind == 0 ? (dd0 - 127 < 0 || dd0 + 127 >= w0)
+                                          : (dd0 - 127 < 0);
       if (need_mask) {
         const int dd = dd0 + row;  // i - j = dd - col
 #pragma unroll
         for (int col = 0; col < 128; ++col) {
           const int rel = dd - col;
-          const bool keep = remote ? (rel >= w0) : (rel >= 0 && rel < w0);
+          const bool keep = mkind == 1 ? (rel >= w0) : mkind == 0 ? (rel >= 0 && rel < w0) : (rel >= 0);
           if (!keep) x[col] = -INFINITY;
         }
       }
@@ -478,13 +504,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const int i = mb * kBM + row;  // row of this chunk's Q / O / LSE
-      const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      const float inv = (l_sum > 0.f && npass > 0) ? 1.f / l_sum : 0.f;
       __nv_bfloat16* orow = args.o + (((size_t)b * args.Lq + i) * args.Hq + hq) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
-        tmem_ld32(o_addr + c * 32, ov);
-        tmem_ld_wait(ov);
+        if (npass > 0) {
+          tmem_ld32(o_addr + c * 32, ov);
+          tmem_ld_wait(ov);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = 0u;  // no key: O = 0, LSE = -inf
+        }
         uint32_t w[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -497,7 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (args.lse != nullptr && i < args.Lq) {
         const float m = (m_used == -INFINITY) ? 0.f : m_used;
-        args.lse[((size_t)b * args.Hq + hq) * args.Lq + i] = (m + __log2f(l_sum)) * 0.69314718055994531f;
+        args.lse[((size_t)b * args.Hq + hq) * args.Lq + i] =
+            l_sum > 0.f ? (m + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
       }
     }
   }

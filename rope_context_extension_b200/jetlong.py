@@ -18,7 +18,7 @@ __all__ = [
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
-    "jl_bifocal_prefill_chunk", "EXPORTED_SYMBOLS",
+    "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes", "jl_bifocal_prefill_ie", "EXPORTED_SYMBOLS",
 ]
 
 JL_QSHIFT_NONE = 0
@@ -28,7 +28,8 @@ EXPORTED_SYMBOLS = (
     "jl_status_string", "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes",
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
     "jl_prefill_attention", "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append",
-    "jl_prefill_chunk_workspace_bytes", "jl_bifocal_prefill_chunk",
+    "jl_prefill_chunk_workspace_bytes", "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes",
+    "jl_bifocal_prefill_ie",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +87,10 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_prefill_chunk.argtypes = [c_p, c_p, c_p, c_i64, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_i,
                                            c_d, c_f, c_i, c_p, c_sz, c_p, c_p]
     L.jl_bifocal_prefill_chunk.restype = c_i
+    L.jl_prefill_ie_workspace_bytes.argtypes = [c_i, c_i, c_i, c_i, c_i, c_i]
+    L.jl_prefill_ie_workspace_bytes.restype = c_sz
+    L.jl_bifocal_prefill_ie.argtypes = list(L.jl_bifocal_prefill.argtypes)
+    L.jl_bifocal_prefill_ie.restype = c_i
     _lib = L
     return L
 
@@ -307,3 +312,29 @@ def jl_bifocal_prefill_chunk(q, k_cache, v_cache, o, lse, *, q_offset: int, w0: 
                                         float(softmax_scale), int(mode), _ptr(workspace), ws_bytes, _ptr(dev_error),
                                         _stream(stream))
     _check(st, "jl_bifocal_prefill_chunk")
+
+
+def jl_prefill_ie_workspace_bytes(B: int, L: int, Hq: int, Hkv: int, head_dim: int,
+                                  mode: int = JL_QSHIFT_SELF_EXTEND) -> int:
+    return int(lib().jl_prefill_ie_workspace_bytes(B, L, Hq, Hkv, head_dim, mode))
+
+
+def jl_bifocal_prefill_ie(q, k, v, o, lse, *, w0: int, w_pretrained: int, rope_base: float,
+                          softmax_scale: float = 0.0, mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None,
+                          dev_error=None, stream=None):
+    """The pages' three-call inclusion-exclusion prefill (unfused), same tensors as
+    jl_bifocal_prefill; workspace of jl_prefill_ie_workspace_bytes(...) bytes."""
+    import torch
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _check_tensor(q, "q", torch.bfloat16)
+    _check_tensor(k, "k", torch.bfloat16, (B, L, Hkv, D))
+    _check_tensor(v, "v", torch.bfloat16, (B, L, Hkv, D))
+    _check_tensor(o, "o", torch.bfloat16, (B, L, Hq, D))
+    if lse is not None:
+        _check_tensor(lse, "lse", torch.float32, (B, Hq, L))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().jl_bifocal_prefill_ie(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, L, Hq, Hkv, D, int(w0),
+                                     int(w_pretrained), float(rope_base), float(softmax_scale), int(mode),
+                                     _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream))
+    _check(st, "jl_bifocal_prefill_ie")
