@@ -255,6 +255,31 @@ int jl_rope_append(const void* q_raw, const void* k_raw, const void* v_new, cons
                    double rope_base, int* dev_error, void* stream);
 
 /*
+ * Decode over one key range of a longer sequence (sequence-split decode across
+ * GPUs): cache rows 0 .. key_count - 1 hold the keys at positions key_offset ..
+ * key_offset + key_count - 1 of a sequence of total length total_len, whose new
+ * query sits at position total_len - 1; G, the query shift and the band come
+ * from total_len.  Writes this range's softmax-normalised o [B, Hq, D] (bf16)
+ * and lse [B, Hq] (fp32, required for the combine).  key_offset + key_count
+ * <= total_len; key_count <= cache_len.  Workspace as
+ * jl_decode_workspace_bytes(B, key_count, ...).  Launches one kernel.
+ */
+int jl_bifocal_decode_range(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len,
+                            int key_offset, int key_count, int total_len, void* o, float* lse, int B, int Hq, int Hkv,
+                            int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale, int mode,
+                            void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
+
+/*
+ * Log-sum-exp combine of `parts` partial decode results over disjoint key
+ * ranges (e.g. gathered from the GPUs of a sequence-split decode):
+ * o_parts [parts, B, Hq, D] bf16 and lse_parts [parts, B, Hq] fp32 (device),
+ * o [B, Hq, D] = sum_r exp(lse_r - M) o_r / sum_r exp(lse_r - M),
+ * lse [B, Hq] = M + ln sum_r exp(lse_r - M) (may be NULL).  One launch.
+ */
+int jl_decode_combine(const void* o_parts, const float* lse_parts, int parts, void* o, float* lse, int B, int Hq,
+                      int head_dim, void* stream);
+
+/*
  * jl_bifocal_decode without a workspace argument, for callers that cannot
  * allocate device memory (e.g. a plugin inside an inference engine whose
  * device memory is wholly owned by the host framework's pool, or a serving

@@ -313,6 +313,32 @@ def decode(q, k_cache, v_cache, p: BifocalParams):
     return o, lse
 
 
+def decode_key_range(q, k_cache, v_cache, p: BifocalParams, key_begin: int, key_end: int):
+    """Decode (query at p.L - 1) restricted to keys [key_begin, key_end).
+
+    The scores are the definition's (``bifocal_scores`` with G from p.L); only
+    the softmax is taken over the sub-range, giving that range's normalised
+    output and LSE (the partial result of a sequence-split decode).
+    q: [B, Hq, d]; caches [B, >= p.L, Hkv, d].  Returns O [B, Hq, d], LSE [B, Hq].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    Hkv = np.shape(k_cache)[2]
+    r = Hq // Hkv
+    o = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        for g in range(Hkv):
+            kb = np.asarray(k_cache[b, :p.L, g, :], dtype=np.float64)
+            vb = np.asarray(v_cache[b, key_begin:key_end, g, :], dtype=np.float64)
+            heads = list(range(g * r, (g + 1) * r))
+            s = bifocal_scores(q[b, heads, :], np.full(r, p.L - 1), kb, p)[:, key_begin:key_end]
+            ob, lb = softmax_rows(s, vb)
+            o[b, heads] = ob
+            lse[b, heads] = lb
+    return o, lse
+
+
 # ---------------------------------------------------------------------------
 # Second formulation: inclusion-exclusion merge of three masked softmaxes
 # ---------------------------------------------------------------------------

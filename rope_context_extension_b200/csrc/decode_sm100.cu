@@ -129,15 +129,20 @@ __global__ void __maxnreg__(168)
       L = L < 1 ? 1 : (int)args.cache_len;
     }
   }
-  const int G = (int)group_size(L, args.w_pretrained);
-  const bool all_local = jl::all_local(L, args.w0, G);
-  const int64_t dq = query_remote(L - 1, G, query_shift(args.w0, G, args.qshift)) - (L - 1);
+  // Key row j of this call sits at position j + key_off; the query at Lpos - 1
+  // (Lpos = the sequence's total length; a sequence-split decode gives each
+  // GPU one key range of the cache and the global length).
+  const int key_off = args.key_off;
+  const int Lpos = args.L_total > 0 ? args.L_total : L;
+  const int G = (int)group_size(Lpos, args.w_pretrained);
+  const bool all_local = jl::all_local(Lpos, args.w0, G);
+  const int64_t dq = query_remote(Lpos - 1, G, query_shift(args.w0, G, args.qshift)) - (Lpos - 1);
   const uint32_t g_magic = G < 16 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)G - 1) / (uint64_t)G) : 0u;
   const int ntiles_b = (L + kDecKeys - 1) / kDecKeys;
   const int t_begin = (int)(((int64_t)split * ntiles_b) / args.splits);
   const int t_end = (int)(((int64_t)(split + 1) * ntiles_b) / args.splits);
   const int ntile = t_end - t_begin;  // may be 0 for short sequences of a varlen batch
-  const int local_from = all_local ? 0 : L - args.w0;  // keys j >= local_from are local
+  const int local_from = all_local ? 0 : Lpos - args.w0 - key_off;  // rows j >= local_from are local
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -165,7 +170,7 @@ __global__ void __maxnreg__(168)
       } else if (row < 18) {
         turns = -(double)(q64 + (row - 16) - 64);  // -(dk(j0 + 64) - dk(j0))
       } else {
-        const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18);
+        const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18) + key_off;  // position
         turns = (double)(dq - (j0 / G - j0));
       }
       double sn, cs;
@@ -270,8 +275,8 @@ __global__ void __maxnreg__(168)
 
   // Group arithmetic of this warp's tile start j0, advanced by 64 keys per
   // tile without divisions: j0 = qd G + rm.
-  int j0 = t_begin * kDecKeys + 16 * warp;
-  int qd = j0 / G, rm = j0 - qd * G;
+  int j0 = t_begin * kDecKeys + 16 * warp;  // row in this call's cache
+  int qd = (j0 + key_off) / G, rm = (j0 + key_off) - qd * G;  // of the position j0 + key_off
   const int q64 = kDecKeys / G, r64 = kDecKeys - q64 * G;
   // floor(x / G) for 0 <= x < G + 16 (one multiply-high; exact there)
   auto div_small = [&](int x) -> int {

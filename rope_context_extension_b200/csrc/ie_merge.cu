@@ -1,3 +1,6 @@
+// Log-sum-exp merges: the inclusion-exclusion merge of the three calls of the
+// pages' prefill formulation, and the combine of a sequence-split decode.
+//
 // Inclusion-exclusion merge of the three calls of the pages' prefill
 // formulation (Jet-Long review, "Method"):
 //   O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C),  W_X = exp(LSE_X - M),
@@ -44,7 +47,49 @@ __global__ void __launch_bounds__(256) ie_merge_kernel(const __grid_constant__ M
   if (lane == 0 && a.lse != nullptr) a.lse[lidx] = M + logf(den);
 }
 
+// O = sum_r exp(LSE_r - M) O_r / sum_r exp(LSE_r - M), LSE = M + ln(sum ...):
+// partial results over disjoint key ranges of one query (a sequence-split
+// decode), one warp per (sequence, head).
+template <int D>
+__global__ void __launch_bounds__(256) lse_combine_kernel(const __grid_constant__ CombineArgs a) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rows = a.B * a.Hq;
+  if (row >= rows) return;
+  float M = -INFINITY;
+  for (int r = 0; r < a.R; ++r) M = fmaxf(M, a.lse_parts[(size_t)r * rows + row]);
+  float den = 0.f;
+  for (int r = 0; r < a.R; ++r) {
+    const float l = a.lse_parts[(size_t)r * rows + row];
+    den += l == -INFINITY ? 0.f : expf(l - M);
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  constexpr int kPer = D / 32;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int d = lane + 32 * e;
+    float acc = 0.f;
+    for (int r = 0; r < a.R; ++r) {
+      const float l = a.lse_parts[(size_t)r * rows + row];
+      const float w = l == -INFINITY ? 0.f : expf(l - M);
+      acc += w * __bfloat162float(a.o_parts[((size_t)r * rows + row) * D + d]);
+    }
+    a.o[(size_t)row * D + d] = __float2bfloat16_rn(acc * inv);
+  }
+  if (lane == 0 && a.lse != nullptr) a.lse[row] = M + logf(den);
+}
+
 }  // namespace
+
+cudaError_t launch_lse_combine(const CombineArgs& a, int D, cudaStream_t stream) {
+  const int rows = a.B * a.Hq;
+  const int blocks = (rows * 32 + 255) / 256;
+  if (D == 128)
+    lse_combine_kernel<128><<<blocks, 256, 0, stream>>>(a);
+  else
+    lse_combine_kernel<64><<<blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_ie_merge(const MergeArgs& a, int D, cudaStream_t stream) {
   const int64_t rows = (int64_t)a.B * a.L * a.Hq;

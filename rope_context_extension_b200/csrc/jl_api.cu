@@ -445,8 +445,9 @@ namespace {
 int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len,
                   const int32_t* seq_lens, int L, void* o, float* lse, int B, int Hq, int Hkv, int D, int w0,
                   int w_pretrained, double rope_base, float softmax_scale, int mode, void* workspace,
-                  size_t workspace_bytes, int* dev_error, void* stream) {
-  int st = common_checks(B, L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+                  size_t workspace_bytes, int* dev_error, void* stream, int key_off = 0, int L_total = 0) {
+  int st = common_checks(B, L_total > 0 ? L_total : L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
+  if (st == JL_OK && L < 1) st = JL_ERR_INVALID_ARG;
   if (st != JL_OK) return st;
   if (!q || !k_cache || !v_cache || !o) return JL_ERR_INVALID_ARG;
   if (cache_len < L || cache_len > (int64_t)1 << 31) return JL_ERR_INVALID_ARG;
@@ -476,6 +477,8 @@ int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64
   a.part_o = reinterpret_cast<float*>(ws + lay.o);
   a.dev_error = dev_error;
   a.seq_lens = seq_lens;
+  a.key_off = key_off;
+  a.L_total = L_total;
   a.B = B;
   a.L = L;
   a.Hq = Hq;
@@ -509,6 +512,35 @@ int jl_bifocal_decode_varlen(const void* q, const void* k_cache, const void* v_c
   if (seq_lens == nullptr) return JL_ERR_INVALID_ARG;
   return decode_launch(q, k_cache, v_cache, cache_len, seq_lens, max_len, o, lse, B, Hq, Hkv, head_dim, w0,
                        w_pretrained, rope_base, softmax_scale, mode, workspace, workspace_bytes, dev_error, stream);
+}
+
+int jl_bifocal_decode_range(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len,
+                            int key_offset, int key_count, int total_len, void* o, float* lse, int B, int Hq, int Hkv,
+                            int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale, int mode,
+                            void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
+  if (key_offset < 0 || key_count < 1 || total_len < 1) return JL_ERR_INVALID_ARG;
+  if ((int64_t)key_offset + key_count > total_len || key_count > cache_len) return JL_ERR_INVALID_ARG;
+  return decode_launch(q, k_cache, v_cache, cache_len, nullptr, key_count, o, lse, B, Hq, Hkv, head_dim, w0,
+                       w_pretrained, rope_base, softmax_scale, mode, workspace, workspace_bytes, dev_error, stream,
+                       key_offset, total_len);
+}
+
+int jl_decode_combine(const void* o_parts, const float* lse_parts, int parts, void* o, float* lse, int B, int Hq,
+                      int head_dim, void* stream) {
+  if (parts < 1 || B < 1 || Hq < 1 || !o_parts || !lse_parts || !o) return JL_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return JL_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(o) || ((uintptr_t)lse_parts & 3u) || (lse && ((uintptr_t)lse & 3u)))
+    return JL_ERR_ALIGNMENT;
+  jl::CombineArgs a;
+  a.o_parts = reinterpret_cast<const __nv_bfloat16*>(o_parts);
+  a.lse_parts = lse_parts;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.R = parts;
+  a.B = B;
+  a.Hq = Hq;
+  if (jl::launch_lse_combine(a, head_dim, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
 }
 
 int jl_rope_append(const void* q_raw, const void* k_raw, const void* v_new, const int32_t* positions, void* q_out,

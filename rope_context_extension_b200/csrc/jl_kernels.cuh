@@ -56,6 +56,8 @@ struct DecodeArgs {
   const int* seq_lens;     // [B] per-sequence L_b (device), or null: every L_b = L
   int B, L, Hq, Hkv, r;    // L: the common length, or the largest L_b
   int64_t cache_len;       // rows of the cache (bound on L_b)
+  int key_off;             // position of cache row 0 (a key range of a longer sequence), else 0
+  int L_total;             // that sequence's total length (query at L_total - 1), or 0: = L
   int splits;              // CTAs per (batch, KV head); each covers a share of its sequence's tiles
   int w0, w_pretrained, qshift;
   float scale_log2;
@@ -77,6 +79,16 @@ struct MergeArgs {
   int B, L, Hq;
 };
 cudaError_t launch_ie_merge(const MergeArgs& a, int D, cudaStream_t stream);
+
+// Log-sum-exp combine of R partial decode results over disjoint key ranges.
+struct CombineArgs {
+  const __nv_bfloat16* o_parts;  // [R, B, Hq, D]
+  const float* lse_parts;        // [R, B, Hq]
+  __nv_bfloat16* o;              // [B, Hq, D]
+  float* lse;                    // [B, Hq] or null
+  int R, B, Hq;
+};
+cudaError_t launch_lse_combine(const CombineArgs& a, int D, cudaStream_t stream);
 
 // Base RoPE of one new token per sequence and its append to the KV cache.
 struct AppendArgs {

@@ -18,7 +18,8 @@ __all__ = [
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
-    "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes", "jl_bifocal_prefill_ie", "EXPORTED_SYMBOLS",
+    "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes", "jl_bifocal_prefill_ie", "jl_bifocal_decode_range",
+    "jl_decode_combine", "EXPORTED_SYMBOLS",
 ]
 
 JL_QSHIFT_NONE = 0
@@ -29,7 +30,7 @@ EXPORTED_SYMBOLS = (
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
     "jl_prefill_attention", "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append",
     "jl_prefill_chunk_workspace_bytes", "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes",
-    "jl_bifocal_prefill_ie",
+    "jl_bifocal_prefill_ie", "jl_bifocal_decode_range", "jl_decode_combine",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +92,11 @@ def lib() -> ctypes.CDLL:
     L.jl_prefill_ie_workspace_bytes.restype = c_sz
     L.jl_bifocal_prefill_ie.argtypes = list(L.jl_bifocal_prefill.argtypes)
     L.jl_bifocal_prefill_ie.restype = c_i
+    L.jl_bifocal_decode_range.argtypes = [c_p, c_p, c_p, c_i64, c_i, c_i, c_i, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i,
+                                          c_d, c_f, c_i, c_p, c_sz, c_p, c_p]
+    L.jl_bifocal_decode_range.restype = c_i
+    L.jl_decode_combine.argtypes = [c_p, c_p, c_i, c_p, c_p, c_i, c_i, c_i, c_p]
+    L.jl_decode_combine.restype = c_i
     _lib = L
     return L
 
@@ -338,3 +344,39 @@ def jl_bifocal_prefill_ie(q, k, v, o, lse, *, w0: int, w_pretrained: int, rope_b
                                      int(w_pretrained), float(rope_base), float(softmax_scale), int(mode),
                                      _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream))
     _check(st, "jl_bifocal_prefill_ie")
+
+
+def jl_bifocal_decode_range(q, k_cache, v_cache, o, lse, *, key_offset: int, key_count: int, total_len: int, w0: int,
+                            w_pretrained: int, rope_base: float, softmax_scale: float = 0.0,
+                            mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None, dev_error=None, stream=None):
+    """Decode over cache rows holding positions key_offset..key_offset+key_count-1 of a
+    sequence of total length total_len; o [B, Hq, D] bf16 and lse [B, Hq] fp32 are this
+    range's normalised partial result."""
+    import torch
+    B, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    _check_tensor(q, "q", torch.bfloat16)
+    _check_tensor(k_cache, "k_cache", torch.bfloat16)
+    _check_tensor(v_cache, "v_cache", torch.bfloat16, tuple(k_cache.shape))
+    _check_tensor(o, "o", torch.bfloat16, (B, Hq, D))
+    _check_tensor(lse, "lse", torch.float32, (B, Hq))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().jl_bifocal_decode_range(_ptr(q), _ptr(k_cache), _ptr(v_cache), Lmax, int(key_offset), int(key_count),
+                                       int(total_len), _ptr(o), _ptr(lse), B, Hq, Hkv, D, int(w0), int(w_pretrained),
+                                       float(rope_base), float(softmax_scale), int(mode), _ptr(workspace), ws_bytes,
+                                       _ptr(dev_error), _stream(stream))
+    _check(st, "jl_bifocal_decode_range")
+
+
+def jl_decode_combine(o_parts, lse_parts, o, lse, stream=None):
+    """Log-sum-exp combine of partial results: o_parts [R, B, Hq, D] bf16,
+    lse_parts [R, B, Hq] fp32 (CUDA) into o [B, Hq, D] and lse [B, Hq] (or None)."""
+    import torch
+    R, B, Hq, D = o_parts.shape
+    _check_tensor(o_parts, "o_parts", torch.bfloat16)
+    _check_tensor(lse_parts, "lse_parts", torch.float32, (R, B, Hq))
+    _check_tensor(o, "o", torch.bfloat16, (B, Hq, D))
+    if lse is not None:
+        _check_tensor(lse, "lse", torch.float32, (B, Hq))
+    st = lib().jl_decode_combine(_ptr(o_parts), _ptr(lse_parts), R, _ptr(o), _ptr(lse), B, Hq, D, _stream(stream))
+    _check(st, "jl_decode_combine")
