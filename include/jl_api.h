@@ -280,6 +280,14 @@ int jl_decode_combine(const void* o_parts, const float* lse_parts, int parts, vo
                       int head_dim, void* stream);
 
 /*
+ * Diagnostic: evaluates, on the device, the FMA-pipe exponential that the
+ * prefill softmax uses for part of each row (Cody-Waite reduction plus a fitted
+ * degree-3 polynomial) and CUDA's exp2f on the same n inputs (device arrays),
+ * so its error can be checked.  Not part of the attention path.
+ */
+int jl_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, void* stream);
+
+/*
  * jl_bifocal_decode without a workspace argument, for callers that cannot
  * allocate device memory (e.g. a plugin inside an inference engine whose
  * device memory is wholly owned by the host framework's pool, or a serving

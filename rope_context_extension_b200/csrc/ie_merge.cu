@@ -79,7 +79,29 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const __grid_constant_
   if (lane == 0 && a.lse != nullptr) a.lse[row] = M + logf(den);
 }
 
+// Evaluates the FMA-pipe exponential used by the prefill softmax next to CUDA's
+// exp2f on the same inputs (a check of the polynomial, not a hot path).
+__global__ void exp2_poly_check_kernel(const float* x, float* y_poly, float* y_ref, int n) {
+  const int i2 = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i2 >= n) return;
+  const float a = x[i2], b = (i2 + 1 < n) ? x[i2 + 1] : 0.f;
+  float p0, p1;
+  f2_unpack(ex2_poly2(f2_pack(a, b)), p0, p1);
+  y_poly[i2] = p0;
+  y_ref[i2] = exp2f(a);
+  if (i2 + 1 < n) {
+    y_poly[i2 + 1] = p1;
+    y_ref[i2 + 1] = exp2f(b);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream) {
+  const int pairs = (n + 1) / 2;
+  exp2_poly_check_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y_poly, y_ref, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_lse_combine(const CombineArgs& a, int D, cudaStream_t stream) {
   const int rows = a.B * a.Hq;

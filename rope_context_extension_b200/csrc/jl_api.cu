@@ -543,6 +543,13 @@ int jl_decode_combine(const void* o_parts, const float* lse_parts, int parts, vo
   return JL_OK;
 }
 
+int jl_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, void* stream) {
+  if (!x || !y_poly || !y_ref || n < 1) return JL_ERR_INVALID_ARG;
+  if (jl::launch_exp2_poly_check(x, y_poly, y_ref, n, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
+}
+
 int jl_rope_append(const void* q_raw, const void* k_raw, const void* v_new, const int32_t* positions, void* q_out,
                    void* k_cache, void* v_cache, int64_t cache_len, int B, int Hq, int Hkv, int head_dim,
                    double rope_base, int* dev_error, void* stream) {

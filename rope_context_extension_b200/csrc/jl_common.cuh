@@ -280,4 +280,27 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// 2^x for two values at once on the FMA / ALU pipes (x <= 128): Cody-Waite range
+// reduction 2^x = 2^n * 2^f, n = floor(x), f in [0, 1) (Cody and Waite, Software
+// Manual for the Elementary Functions), and p(f) = 1 + f (c1 + f (c2 + f c3)), a
+// degree-3 minimax fit of 2^f with p(0) = 1 pinned (csrc/exp2_poly_fit.py; max
+// relative error 8.6e-5).  x <= -127 gives exactly 0.  Used for part of the
+// softmax exponentials so that fewer of them queue on the MUFU.
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t xv) {
+  float x0, x1;
+  f2_unpack(xv, x0, x1);
+  x0 = fmaxf(x0, -127.f);
+  x1 = fmaxf(x1, -127.f);
+  const float n0 = floorf(x0), n1 = floorf(x1);
+  const uint64_t f = f2_sub(f2_pack(x0, x1), f2_pack(n0, n1));
+  uint64_t p = f2_fma(f, f2_pack(0.0770670399f, 0.0770670399f), f2_pack(0.227644995f, 0.227644995f));
+  p = f2_fma(f, p, f2_pack(0.695116758f, 0.695116758f));
+  p = f2_fma(f, p, f2_pack(1.f, 1.f));
+  float p0, p1;
+  f2_unpack(p, p0, p1);
+  p0 = __int_as_float(__float_as_int(p0) + ((int)n0 << 23));
+  p1 = __int_as_float(__float_as_int(p1) + ((int)n1 << 23));
+  return f2_pack(p0, p1);
+}
+
 }  // namespace jl

@@ -40,8 +40,14 @@ constexpr int kBN = 128;  // keys per tile
 constexpr int kStages = 2;
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
-constexpr int kLowRegs = 104;      // warpgroup 0: TMA producer, MMA issuer
+constexpr int kLowRegs = 104;     // warpgroup 0: TMA producer, MMA issuer
 constexpr int kHighRegs = 200;    // warpgroups 1-2: softmax
+// kPolyEvery > 0 sends one pair of exponentials in every kPolyEvery to the FMA
+// pipe (ex2_poly2) instead of the MUFU.  Measured at the 128K workload with
+// one pair in four: 879 TFLOP/s against 1000-1040 with all exponentials on the
+// MUFU — the softmax is bound by issue and latency, not by MUFU throughput —
+// so it is off.
+constexpr int kPolyEvery = 0;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kChunkBytes = 128 * 128;  // one 128-row x 128-byte swizzled slab
 
@@ -87,7 +93,6 @@ static_assert(kNumBars * 8 <= 192, "barrier block overflow");
 // remote passes on nb_rem_max, ..., 0 (the blocks with a pair i - j >= w0).
 struct Sched {
   int n_loc, n_rem, nb_max, nb_rem_max;
-  int kind;
 };
 
 __device__ __forceinline__ int floor_div128(int x) { return x >= 0 ? x / 128 : -((127 - x) / 128); }
@@ -97,9 +102,9 @@ __device__ __forceinline__ int floor_div128(int x) { return x >= 0 ? x / 128 : -
 // "Method"): kWindowBase (A: pairs with 0 <= i - j < w0, base rows),
 // kCausalRemote (B: every causal pair, corrected rows), kWindowRemote (C: the
 // window of A, corrected rows).
-__device__ __forceinline__ Sched make_sched(int off, int w0, bool all_local, int kind) {
+template <int kind>
+__device__ __forceinline__ Sched make_sched(int off, int w0, bool all_local) {
   Sched s;
-  s.kind = kind;
   s.nb_max = (off + 127) / 128;  // last block holding a causal key
   if (kind == kCausalRemote) {
     s.n_loc = 0;
@@ -128,13 +133,15 @@ __device__ __forceinline__ int pass_block(const Sched& s, int p) {
   return p < s.n_loc ? s.nb_max - p : s.nb_rem_max - (p - s.n_loc);
 }
 // Does pass p read the corrected (remote-position) Q / K rows?
+template <int kind>
 __device__ __forceinline__ bool pass_remote_ops(const Sched& s, int p) {
-  return s.kind == kBifocal ? p >= s.n_loc : (s.kind != kWindowBase);
+  return kind == kBifocal ? p >= s.n_loc : (kind != kWindowBase);
 }
 // Which pairs of the tile pass p keeps: 0 band (0 <= i-j < w0), 1 beyond the
 // band (i-j >= w0), 2 every causal pair (i-j >= 0).
+template <int kind>
 __device__ __forceinline__ int pass_mask_kind(const Sched& s, int p) {
-  if (s.kind == kCausalRemote) return 2;
+  if (kind == kCausalRemote) return 2;
   return p < s.n_loc ? 0 : 1;
 }
 
@@ -148,7 +155,7 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-template <int D, bool kSplit>
+template <int D, bool kSplit, int kKind>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
@@ -203,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
   const int off = args.q_off + mb * kBM;  // position of this block's first query
-  const Sched sc = make_sched(off, args.w0, args.all_local != 0, args.kind);
+  const Sched sc = make_sched<kKind>(off, args.w0, args.all_local != 0);
   const int npass = sc.n_loc + sc.n_rem;
   const bool q_switch = sc.n_loc > 0 && sc.n_rem > 0;
   const int w0 = args.w0;
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         hq0 + hh, mb * kBM, b);
       };
       // A query block with no pass (a window call with w0 = 0) loads nothing.
-      if (npass > 0) load_q(pass_remote_ops(sc, 0));
+      if (npass > 0) load_q(pass_remote_ops<kKind>(sc, 0));
       int q_loads = npass > 0 ? 1 : 0;
       int k_last = -1, v_last = -1;  // last passes whose K / V copies were issued
       bool ok = true;
@@ -256,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (uint32_t)(p / kStages) & 1u;
         const int sv = p % C::kVStages;
         const uint32_t phv = (uint32_t)(p / C::kVStages) & 1u;
-        const bool remote = pass_remote_ops(sc, p);
+        const bool remote = pass_remote_ops<kKind>(sc, p);
         const int nb = pass_block(sc, p);
         if (q_switch && p == sc.n_loc) {
           if (!(ok = mbar_wait(bar(kQEmpty), 0, abort_flag, args.dev_error))) break;
@@ -310,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t qa = sbase + C::kQOff + h * C::kTileBytes;
         const uint32_t ka = sbase + C::kKOff + s * C::kKSlots * C::kTileBytes;
-        const bool remote = pass_remote_ops(sc, p);
+        const bool remote = pass_remote_ops<kKind>(sc, p);
         const uint32_t id_s = remote ? id_s_rem : id_s_loc;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -401,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int mkind = pass_mask_kind(sc, p);
+      const int mkind = pass_mask_kind<kKind>(sc, p);
       const int dd0 = off - 128 * pass_block(sc, p);  // i - j at row 0, column 0
 
       uint32_t sr[4][32];
@@ -465,10 +472,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          float e0, e1;
-          f2_unpack(f2_fma(f2_pack(x[half * 64 + 2 * k], x[half * 64 + 2 * k + 1]), sc2, nm2), e0, e1);
-          const float p0 = ex2_approx(e0);
-          const float p1 = ex2_approx(e1);
+          const uint64_t ev = f2_fma(f2_pack(x[half * 64 + 2 * k], x[half * 64 + 2 * k + 1]), sc2, nm2);
+          float p0, p1;
+          if (kPolyEvery > 0 && (k % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+            f2_unpack(ex2_poly2(ev), p0, p1);  // on the FMA pipe
+          } else {
+            float e0, e1;
+            f2_unpack(ev, e0, e1);
+            p0 = ex2_approx(e0);  // on the MUFU
+            p1 = ex2_approx(e1);
+          }
           acc[k & 1] = f2_add(acc[k & 1], f2_pack(p0, p1));
           pk[k] = pack_bf16x2(p0, p1);
         }
@@ -509,17 +522,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
-        if (npass > 0) {
-          tmem_ld32(o_addr + c * 32, ov);
-          tmem_ld_wait(ov);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) ov[k] = 0u;  // no key: O = 0, LSE = -inf
-        }
+        tmem_ld32(o_addr + c * 32, ov);  // (never written when npass == 0; inv is 0 then)
+        tmem_ld_wait(ov);
         uint32_t w[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          w[k] = pack_bf16x2(__uint_as_float(ov[2 * k]) * inv, __uint_as_float(ov[2 * k + 1]) * inv);
+          w[k] = npass > 0 ? pack_bf16x2(__uint_as_float(ov[2 * k]) * inv, __uint_as_float(ov[2 * k + 1]) * inv)
+                           : 0u;  // no key at all: O = 0, LSE = -inf
         if (i < args.Lq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
@@ -542,11 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
-template <int D, bool kSplit>
+template <int D, bool kSplit, int kKind>
 cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
                              const CUtensorMap& tm_kr_lo, const PrefillArgs& a, cudaStream_t stream) {
-  auto k = bifocal_prefill_kernel<D, kSplit>;
+  auto k = bifocal_prefill_kernel<D, kSplit, kKind>;
   // The setmaxnreg split inside the kernel assumes the launch register count.
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, k);
@@ -559,6 +568,24 @@ cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, 
   return cudaGetLastError();
 }
 
+template <int D, bool kSplit>
+cudaError_t launch_prefill_kind(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
+                                const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
+                                const CUtensorMap& tm_kr_lo, const PrefillArgs& a, cudaStream_t stream) {
+  switch (a.kind) {
+    case kWindowBase:
+      return launch_prefill_t<D, kSplit, kWindowBase>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
+    case kCausalRemote:
+      return launch_prefill_t<D, kSplit, kCausalRemote>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a,
+                                                        stream);
+    case kWindowRemote:
+      return launch_prefill_t<D, kSplit, kWindowRemote>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a,
+                                                        stream);
+    default:
+      return launch_prefill_t<D, kSplit, kBifocal>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
@@ -566,10 +593,10 @@ cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, co
                            const CUtensorMap& tm_kr_lo, const PrefillArgs& a, int D, bool split,
                            cudaStream_t stream) {
   if (D == 128)
-    return split ? launch_prefill_t<128, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
-                 : launch_prefill_t<128, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
-  return split ? launch_prefill_t<64, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
-               : launch_prefill_t<64, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
+    return split ? launch_prefill_kind<128, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
+                 : launch_prefill_kind<128, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
+  return split ? launch_prefill_kind<64, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
+               : launch_prefill_kind<64, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
 }
 
 }  // namespace jl
