@@ -9,9 +9,11 @@
 // dk(j) = f(j) - j.
 //
 // Split-KV layout: grid (splits, Hkv, B); each CTA streams a contiguous run of
-// 64-key tiles of one KV head through a 3-stage TMA ring (128-byte swizzled so
-// ldmatrix is conflict-free) and scores all r = Hq / Hkv query heads of that KV
-// head at once with mma.sync m16n8k16 (heads on the M axis, 16 keys per warp).
+// tiles (16 keys per consumer warp) of one KV head through a TMA ring (128-byte
+// swizzled so ldmatrix is conflict-free) and scores all r = Hq / Hkv query
+// heads of that KV head at once with mma.sync m16n8k16 (heads on the M axis,
+// 16 keys per warp).  The base query's A fragments sit in shared memory (the
+// same for every warp), which keeps the consumers at 164 registers.
 //
 // Correction rotation of keys, per warp tile of 16 keys starting at j0:
 //   dk(j) = dk(j0) - e(j) with e(j) in [0, 15]; the query side carries
@@ -31,9 +33,28 @@ namespace jl {
 
 namespace {
 
-constexpr int kDecKeys = 64;   // keys per stage
-constexpr int kDecStages = 3;
-constexpr int kDecThreads = 160;  // 4 consumer warps + 1 TMA warp
+// Consumer warps per CTA (16 keys each per stage), ring depth and register cap.
+// The register file is split evenly over the four SM sub-partitions (16384
+// registers each) and a CTA's warps are dealt out over them, so at 168
+// registers a sub-partition holds three warps: one CTA of 11 consumer warps +
+// the TMA warp per SM (two 176-key stages, 2 x 88 KB).  The consumers are
+// bound by the latency of the in-register correction, so warps per SM is what
+// counts: measured at B 8 / 128K, 11 warps in one CTA stream the cache about 8%
+// faster than two CTAs of 4 (and 10% faster at B 1).
+#ifndef JL_DEC_WARPS
+#define JL_DEC_WARPS 11
+#endif
+#ifndef JL_DEC_STAGES
+#define JL_DEC_STAGES 2
+#endif
+#ifndef JL_DEC_MAXNREG
+#define JL_DEC_MAXNREG 168
+#endif
+constexpr int kDecWarps = JL_DEC_WARPS;
+constexpr int kDecKeys = 16 * kDecWarps;  // keys per stage
+constexpr int kDecStages = JL_DEC_STAGES;
+constexpr int kDecThreads = 32 * (kDecWarps + 1);  // consumer warps + 1 TMA warp
+static_assert(kDecWarps >= 1 && kDecWarps <= 11, "consumer warps");
 constexpr int kMaxR = 8;       // query heads per KV head handled (M rows used)
 
 template <int D>
@@ -44,8 +65,9 @@ struct DecCfg {
   static constexpr int kERow = (D / 2 + 8) * 8;        // bytes per E row (padded)
   static constexpr int kEOff = kDecStages * kStageBytes;
   static constexpr int kFOff = kEOff + 16 * kERow;
-  static constexpr int kQ0Off = kFOff + 2 * (D / 2) * 8;  // [4 warps][D/2] initial query factors
-  static constexpr int kBarOff = kQ0Off + 4 * (D / 2) * 8;
+  static constexpr int kQ0Off = kFOff + 2 * (D / 2) * 8;  // [warps][D/2] initial query factors
+  static constexpr int kQBOff = kQ0Off + kDecWarps * (D / 2) * 8;  // [D/16][2][32 lanes] base query fragments
+  static constexpr int kBarOff = kQBOff + (D / 16) * 2 * 32 * 4;
   static constexpr int kSmem = kBarOff + 128 + 1024;
   static constexpr int kNT = D / 8;                    // t values per lane
 };
@@ -95,10 +117,12 @@ __device__ __forceinline__ void rot_split_bf16(uint32_t xw, uint32_t yw, const f
   split_f2_bf16(yr, yh, yl);
 }
 
-__device__ __forceinline__ void named_sync_consumers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_sync_consumers() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecWarps) : "memory");
+}
 
 template <int D>
-__global__ void __maxnreg__(168)
+__global__ void __maxnreg__(JL_DEC_MAXNREG)
     bifocal_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ DecodeArgs args) {
   using C = DecCfg<D>;
@@ -148,27 +172,27 @@ __global__ void __maxnreg__(168)
     *abort_flag = 0;
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 4);
+      mbar_init(empty_bar(s), kDecWarps);
     }
     fence_mbar_init();
   }
   // Correction tables (consumers only use them; everyone helps fill them):
   //   E[e][t]  rotation by -e (e in [0, 16)) applied to keys within a warp tile
   //   F[k][t]  advance of the query factor from one warp tile to the next
-  //            (64 keys later), k = (number of new groups) - floor(64 / G)
+  //            (kDecKeys keys later), k = (number of new groups) - floor(kDecKeys / G)
   //   Q0[w][t] rotation by dq - dk(j0) for warp w's first tile
   float2* E = reinterpret_cast<float2*>(smem + C::kEOff);
   float2* F = reinterpret_cast<float2*>(smem + C::kFOff);
   float2* Q0 = reinterpret_cast<float2*>(smem + C::kQ0Off);
   if (!all_local) {
-    const int q64 = 64 / G;
-    for (int idx = threadIdx.x; idx < 22 * H2; idx += blockDim.x) {
+    const int q64 = kDecKeys / G;
+    for (int idx = threadIdx.x; idx < (18 + kDecWarps) * H2; idx += blockDim.x) {
       const int row = idx / H2, t = idx % H2;
       double turns;
       if (row < 16) {
         turns = -(double)row;
       } else if (row < 18) {
-        turns = -(double)(q64 + (row - 16) - 64);  // -(dk(j0 + 64) - dk(j0))
+        turns = -(double)(q64 + (row - 16) - kDecKeys);  // -(dk(j0 + kDecKeys) - dk(j0))
       } else {
         const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18) + key_off;  // position
         turns = (double)(dq - (j0 / G - j0));
@@ -186,9 +210,23 @@ __global__ void __maxnreg__(168)
       }
     }
   }
+  // The base query as A fragments of mma m16n8k16 (heads on M rows 0-7),
+  // identical for every consumer warp: [k-step][a1 / a3][lane] holds the bf16
+  // pair at dims 16 ks + 2 (lane % 4) (+ 8) of head lane / 4.
+  uint32_t* QB = reinterpret_cast<uint32_t*>(smem + C::kQBOff);
+  for (int idx = threadIdx.x; idx < KS * 2 * 32; idx += blockDim.x) {
+    const int ks = idx / 64, hf = (idx / 32) & 1, l = idx & 31;
+    const int hr = l >> 2;
+    uint32_t w = 0u;
+    if (hr < r) {
+      const __nv_bfloat16* qp = args.q + ((size_t)b * args.Hq + g * r + hr) * D + 16 * ks + 8 * hf + 2 * (l & 3);
+      w = *reinterpret_cast<const uint32_t*>(qp);
+    }
+    QB[idx] = w;
+  }
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == kDecWarps) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&tm_k);
@@ -223,32 +261,22 @@ __global__ void __maxnreg__(168)
   const int c4 = lane & 3;        // column group of the mma fragments
   const int hrow = lane >> 2;     // query head (M row) of this lane
   const bool head_ok = hrow < r;
-  const int hq = g * r + hrow;
 
-  // Base query A fragments (bf16 as given) and the fp32 query copy in the
-  // lane's t-set: t = 16 ks + 2 c4 + {0, 1, 8, 9}, ks < D/32.
-  uint32_t qa_base[KS][2];
+  // The fp32 query copy in the lane's t-set: t = 16 ks + 2 c4 + {0, 1, 8, 9},
+  // ks < D/32 (the base fragments stay in shared memory for local tiles).
   float qre[C::kNT], qim[C::kNT];
-  {
-    const __nv_bfloat16* qp = args.q + ((size_t)b * args.Hq + (head_ok ? hq : 0)) * D;
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const uint32_t w0v = head_ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks + 2 * c4) : 0u;
-      const uint32_t w2v = head_ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks + 8 + 2 * c4) : 0u;
-      qa_base[ks][0] = w0v;
-      qa_base[ks][1] = w2v;
-    }
-#pragma unroll
-    for (int ks = 0; ks < KS2; ++ks) {
-      qre[4 * ks + 0] = bf16lo_to_f32(qa_base[ks][0]);
-      qre[4 * ks + 1] = bf16hi_to_f32(qa_base[ks][0]);
-      qre[4 * ks + 2] = bf16lo_to_f32(qa_base[ks][1]);
-      qre[4 * ks + 3] = bf16hi_to_f32(qa_base[ks][1]);
-      qim[4 * ks + 0] = bf16lo_to_f32(qa_base[ks + KS2][0]);
-      qim[4 * ks + 1] = bf16hi_to_f32(qa_base[ks + KS2][0]);
-      qim[4 * ks + 2] = bf16lo_to_f32(qa_base[ks + KS2][1]);
-      qim[4 * ks + 3] = bf16hi_to_f32(qa_base[ks + KS2][1]);
-    }
+  for (int ks = 0; ks < KS2; ++ks) {
+    const uint32_t x0 = QB[(ks * 2 + 0) * 32 + lane], x1 = QB[(ks * 2 + 1) * 32 + lane];
+    const uint32_t y0 = QB[((ks + KS2) * 2 + 0) * 32 + lane], y1 = QB[((ks + KS2) * 2 + 1) * 32 + lane];
+    qre[4 * ks + 0] = bf16lo_to_f32(x0);
+    qre[4 * ks + 1] = bf16hi_to_f32(x0);
+    qre[4 * ks + 2] = bf16lo_to_f32(x1);
+    qre[4 * ks + 3] = bf16hi_to_f32(x1);
+    qim[4 * ks + 0] = bf16lo_to_f32(y0);
+    qim[4 * ks + 1] = bf16hi_to_f32(y0);
+    qim[4 * ks + 2] = bf16lo_to_f32(y1);
+    qim[4 * ks + 3] = bf16hi_to_f32(y1);
   }
   // q^c = R(dq - dk(j0)) q for this warp's first 16-key tile.
   if (!all_local) {
@@ -273,7 +301,7 @@ __global__ void __maxnreg__(168)
   const float sl2 = args.scale_log2;
   bool ok = true;
 
-  // Group arithmetic of this warp's tile start j0, advanced by 64 keys per
+  // Group arithmetic of this warp's tile start j0, advanced by kDecKeys keys per
   // tile without divisions: j0 = qd G + rm.
   int j0 = t_begin * kDecKeys + 16 * warp;  // row in this call's cache
   int qd = (j0 + key_off) / G, rm = (j0 + key_off) - qd * G;  // of the position j0 + key_off
@@ -362,8 +390,8 @@ __global__ void __maxnreg__(168)
           }
         }
         if (!t_remote) {  // local or straddling: base query, keys as stored
-          const uint32_t alo[4] = {qa_base[kp][0], 0u, qa_base[kp][1], 0u};
-          const uint32_t ahi[4] = {qa_base[kp + KS2][0], 0u, qa_base[kp + KS2][1], 0u};
+          const uint32_t alo[4] = {QB[(kp * 2) * 32 + lane], 0u, QB[(kp * 2 + 1) * 32 + lane], 0u};
+          const uint32_t ahi[4] = {QB[((kp + KS2) * 2) * 32 + lane], 0u, QB[((kp + KS2) * 2 + 1) * 32 + lane], 0u};
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             mma_bf16(sloc[nt], alo, klo[2 * nt], klo[2 * nt + 1]);
@@ -468,9 +496,9 @@ __global__ void __maxnreg__(168)
   l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
   l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
   named_sync_consumers();  // every warp is done with the stage buffers
-  float* mw = reinterpret_cast<float*>(smem);                    // [4][kMaxR]
-  float* lw = mw + 4 * kMaxR;                                    // [4][kMaxR]
-  float* ow = lw + 4 * kMaxR;                                    // [4][kMaxR][D]
+  float* mw = reinterpret_cast<float*>(smem);  // [warps][kMaxR]
+  float* lw = mw + kDecWarps * kMaxR;          // [warps][kMaxR]
+  float* ow = lw + kDecWarps * kMaxR;          // [warps][kMaxR][D]
   if (head_ok && c4 == 0) {
     mw[warp * kMaxR + hrow] = m_used;
     lw[warp * kMaxR + hrow] = l_part;
@@ -486,14 +514,14 @@ __global__ void __maxnreg__(168)
   }
   named_sync_consumers();
   const size_t pbase = (((size_t)b * args.Hkv + g) * args.splits + split) * r;
-  for (int idx = threadIdx.x; idx < r * D; idx += 128) {
+  for (int idx = threadIdx.x; idx < r * D; idx += 32 * kDecWarps) {
     const int h = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, mw[w * kMaxR + h]);
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mw[w * kMaxR + h]);
     float o = 0.f, l = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < kDecWarps; ++w) {
       const float mwv = mw[w * kMaxR + h];
       const float wt = (mwv == -INFINITY) ? 0.f : ex2_approx(mwv - M);
       o += wt * ow[(w * kMaxR + h) * D + d];
@@ -514,7 +542,7 @@ __global__ void __maxnreg__(168)
   if (*ticket_slot == 0) return;
   __threadfence();
   const size_t sbase_p = ((size_t)b * args.Hkv + g) * args.splits;
-  for (int h = warp; h < r; h += 4) {
+  for (int h = warp; h < r; h += kDecWarps) {
     float M = -INFINITY;
     for (int sp = lane; sp < args.splits; sp += 32) M = fmaxf(M, __ldcg(&args.part_ml[(sbase_p + sp) * r + h]).x);
 #pragma unroll
@@ -552,6 +580,8 @@ cudaError_t set_decode_attrs() {
 }
 
 }  // namespace
+
+int decode_tile_keys() { return kDecKeys; }
 
 int decode_ctas_per_sm() {
   static int cached = 0;

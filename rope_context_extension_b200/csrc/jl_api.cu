@@ -90,7 +90,7 @@ int decode_splits_max(int B, int Hkv) {
   return s;
 }
 
-// Split count for one call: whole 64-key tiles per split, and the CTA count
+// Split count for one call: whole decode tiles per split, and the CTA count
 // chosen so the last wave on the GPU is as full as possible (at least four
 // tiles per split so the per-CTA set-up stays small).
 int decode_splits(int B, int Hkv, int ntiles) {
@@ -455,15 +455,16 @@ int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
       (lse && ((uintptr_t)lse & 3u)) || (seq_lens && ((uintptr_t)seq_lens & 3u)))
     return JL_ERR_ALIGNMENT;
-  const int ntiles = (L + 63) / 64;
+  const int tk_keys = jl::decode_tile_keys();
+  const int ntiles = (L + tk_keys - 1) / tk_keys;
   const int splits = decode_splits(B, Hkv, ntiles);
   const DecodeLayout lay = decode_layout(B, Hq, Hkv, D, decode_splits_max(B, Hkv));
   if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
 
   CUtensorMap tk, tv;
-  if (!encode_bf16_4d(&tk, k_cache, D, Hkv, cache_len, B, 64) ||
-      !encode_bf16_4d(&tv, v_cache, D, Hkv, cache_len, B, 64))
+  if (!encode_bf16_4d(&tk, k_cache, D, Hkv, cache_len, B, tk_keys) ||
+      !encode_bf16_4d(&tv, v_cache, D, Hkv, cache_len, B, tk_keys))
     return JL_ERR_CUDA;
 
   DecodeArgs a;

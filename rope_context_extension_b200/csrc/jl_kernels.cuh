@@ -69,6 +69,8 @@ cudaError_t launch_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, cons
                           cudaStream_t stream);
 // Resident decode CTAs per SM (occupancy of the D = 128 kernel, cached).
 int decode_ctas_per_sm();
+// Keys per decode tile (one TMA stage; splits cover whole tiles).
+int decode_tile_keys();
 
 // Inclusion-exclusion merge of three partial prefill outputs.
 struct MergeArgs {
