@@ -61,9 +61,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Source files that determine each timed kernel's code and launch shape; a
+# traffic figure is used only while these hash to the value stored with it.
+KERNEL_SOURCES = {
+    "prefill_attention": ["prefill_sm100.cu", "jl_common.cuh", "jl_kernels.cuh", "jl_api.cu"],
+    "decode": ["decode_sm100.cu", "jl_common.cuh", "jl_kernels.cuh", "jl_api.cu"],
+}
+
+
 def load_traffic():
     """Per-launch DRAM bytes of the timed kernels from the committed ncu summary,
-    valid only while the kernel sources hash to the value recorded with them."""
+    each valid only while its kernel's sources hash to the value recorded with it."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return {}
@@ -72,15 +80,15 @@ def load_traffic():
             data = json.load(f)
     except (OSError, ValueError):
         return {}
-    cur = sources_hash()
-    return {k: v for k, v in data.items() if isinstance(v, dict) and v.get("sources") == cur}
+    return {k: v for k, v in data.items()
+            if isinstance(v, dict) and k in KERNEL_SOURCES and v.get("sources") == sources_hash(KERNEL_SOURCES[k])}
 
 
-def sources_hash():
+def sources_hash(files):
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rope_context_extension_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]

@@ -173,10 +173,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int NH = args.nh;
-  const int hq0 = blockIdx.x * NH;
-  const int mb = args.num_mb - 1 - (int)blockIdx.y;  // heaviest blocks first
-  const int b = blockIdx.z;
-  const int kvh = hq0 / args.r;
+  // Work order (CTAs launch in increasing linear index): the CTAs of one KV
+  // head's query heads run together, heaviest query blocks first, so the CTAs
+  // resident at any time stream the same K / V rows and re-read them from L2.
+  const int hpk = args.r / NH;  // CTAs (query-head groups) per KV head and block
+  int lin = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+  const int hg = lin % hpk;
+  lin /= hpk;
+  const int mb = args.num_mb - 1 - lin % args.num_mb;
+  lin /= args.num_mb;
+  const int kvh = lin % args.Hkv;
+  const int b = lin / args.Hkv;
+  const int hq0 = (kvh * hpk + hg) * NH;
   const uint32_t ncols = NH == 2 ? 512u : 256u;
 
   if (threadIdx.x == 0) {
