@@ -176,58 +176,10 @@ __global__ void __maxnreg__(JL_DEC_MAXNREG)
     }
     fence_mbar_init();
   }
-  // Correction tables (consumers only use them; everyone helps fill them):
-  //   E[e][t]  rotation by -e (e in [0, 16)) applied to keys within a warp tile
-  //   F[k][t]  advance of the query factor from one warp tile to the next
-  //            (kDecKeys keys later), k = (number of new groups) - floor(kDecKeys / G)
-  //   Q0[w][t] rotation by dq - dk(j0) for warp w's first tile
-  float2* E = reinterpret_cast<float2*>(smem + C::kEOff);
-  float2* F = reinterpret_cast<float2*>(smem + C::kFOff);
-  float2* Q0 = reinterpret_cast<float2*>(smem + C::kQ0Off);
-  if (!all_local) {
-    const int q64 = kDecKeys / G;
-    for (int idx = threadIdx.x; idx < (18 + kDecWarps) * H2; idx += blockDim.x) {
-      const int row = idx / H2, t = idx % H2;
-      double turns;
-      if (row < 16) {
-        turns = -(double)row;
-      } else if (row < 18) {
-        turns = -(double)(q64 + (row - 16) - kDecKeys);  // -(dk(j0 + kDecKeys) - dk(j0))
-      } else {
-        const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18) + key_off;  // position
-        turns = (double)(dq - (j0 / G - j0));
-      }
-      double sn, cs;
-      sincos(turns * args.theta[t], &sn, &cs);
-      // E and F rows hold (c_t, c_t+1, s_t, s_t+1) for even t; Q0 rows (c_t, s_t)
-      float* dst = row < 16 ? reinterpret_cast<float*>(E) + row * (C::kERow / 4)
-                            : reinterpret_cast<float*>(F) + (row - 16) * D;
-      if (row < 18) {
-        dst[(t >> 1) * 4 + (t & 1)] = (float)cs;
-        dst[(t >> 1) * 4 + 2 + (t & 1)] = (float)sn;
-      } else {
-        Q0[(row - 18) * H2 + t] = make_float2((float)cs, (float)sn);
-      }
-    }
-  }
-  // The base query as A fragments of mma m16n8k16 (heads on M rows 0-7),
-  // identical for every consumer warp: [k-step][a1 / a3][lane] holds the bf16
-  // pair at dims 16 ks + 2 (lane % 4) (+ 8) of head lane / 4.
-  uint32_t* QB = reinterpret_cast<uint32_t*>(smem + C::kQBOff);
-  for (int idx = threadIdx.x; idx < KS * 2 * 32; idx += blockDim.x) {
-    const int ks = idx / 64, hf = (idx / 32) & 1, l = idx & 31;
-    const int hr = l >> 2;
-    uint32_t w = 0u;
-    if (hr < r) {
-      const __nv_bfloat16* qp = args.q + ((size_t)b * args.Hq + g * r + hr) * D + 16 * ks + 8 * hf + 2 * (l & 3);
-      w = *reinterpret_cast<const uint32_t*>(qp);
-    }
-    QB[idx] = w;
-  }
   __syncthreads();
-
   if (warp == kDecWarps) {
     // ------------------------------------------------------------ TMA producer
+    // (starts streaming at once; the consumers build their tables meanwhile)
     if (lane == 0) {
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
@@ -256,6 +208,56 @@ __global__ void __maxnreg__(JL_DEC_MAXNREG)
     }
     return;
   }
+  constexpr int kCons = 32 * kDecWarps;  // consumer threads
+  // Correction tables (the consumers fill and use them):
+  //   E[e][t]  rotation by -e (e in [0, 16)) applied to keys within a warp tile
+  //   F[k][t]  advance of the query factor from one warp tile to the next
+  //            (kDecKeys keys later), k = (number of new groups) - floor(kDecKeys / G)
+  //   Q0[w][t] rotation by dq - dk(j0) for warp w's first tile
+  float2* E = reinterpret_cast<float2*>(smem + C::kEOff);
+  float2* F = reinterpret_cast<float2*>(smem + C::kFOff);
+  float2* Q0 = reinterpret_cast<float2*>(smem + C::kQ0Off);
+  if (!all_local) {
+    const int q64 = kDecKeys / G;
+    for (int idx = threadIdx.x; idx < (18 + kDecWarps) * H2; idx += kCons) {
+      const int row = idx / H2, t = idx % H2;
+      double turns;
+      if (row < 16) {
+        turns = -(double)row;
+      } else if (row < 18) {
+        turns = -(double)(q64 + (row - 16) - kDecKeys);  // -(dk(j0 + kDecKeys) - dk(j0))
+      } else {
+        const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18) + key_off;  // position
+        turns = (double)(dq - (j0 / G - j0));
+      }
+      double sn, cs;
+      sincos(turns * args.theta[t], &sn, &cs);
+      // E and F rows hold (c_t, c_t+1, s_t, s_t+1) for even t; Q0 rows (c_t, s_t)
+      float* dst = row < 16 ? reinterpret_cast<float*>(E) + row * (C::kERow / 4)
+                            : reinterpret_cast<float*>(F) + (row - 16) * D;
+      if (row < 18) {
+        dst[(t >> 1) * 4 + (t & 1)] = (float)cs;
+        dst[(t >> 1) * 4 + 2 + (t & 1)] = (float)sn;
+      } else {
+        Q0[(row - 18) * H2 + t] = make_float2((float)cs, (float)sn);
+      }
+    }
+  }
+  // The base query as A fragments of mma m16n8k16 (heads on M rows 0-7),
+  // identical for every consumer warp: [k-step][a1 / a3][lane] holds the bf16
+  // pair at dims 16 ks + 2 (lane % 4) (+ 8) of head lane / 4.
+  uint32_t* QB = reinterpret_cast<uint32_t*>(smem + C::kQBOff);
+  for (int idx = threadIdx.x; idx < KS * 2 * 32; idx += kCons) {
+    const int ks = idx / 64, hf = (idx / 32) & 1, l = idx & 31;
+    const int hr = l >> 2;
+    uint32_t w = 0u;
+    if (hr < r) {
+      const __nv_bfloat16* qp = args.q + ((size_t)b * args.Hq + g * r + hr) * D + 16 * ks + 8 * hf + 2 * (l & 3);
+      w = *reinterpret_cast<const uint32_t*>(qp);
+    }
+    QB[idx] = w;
+  }
+  named_sync_consumers();
 
   // -------------------------------------------------------------- consumers
   const int c4 = lane & 3;        // column group of the mma fragments
@@ -542,30 +544,40 @@ __global__ void __maxnreg__(JL_DEC_MAXNREG)
   if (*ticket_slot == 0) return;
   __threadfence();
   const size_t sbase_p = ((size_t)b * args.Hkv + g) * args.splits;
+  const int S = args.splits;
+  // Per head: the global max and sum over the splits (lanes over splits), then
+  // each split's weight 2^(m_s - M) / l in shared memory (the stage area is
+  // free); then every consumer thread reduces its (head, dim) outputs over the
+  // splits with independent loads in flight.
+  float* wts = reinterpret_cast<float*>(smem);  // [r][S]
   for (int h = warp; h < r; h += kDecWarps) {
     float M = -INFINITY;
-    for (int sp = lane; sp < args.splits; sp += 32) M = fmaxf(M, __ldcg(&args.part_ml[(sbase_p + sp) * r + h]).x);
+    for (int sp = lane; sp < S; sp += 32) M = fmaxf(M, __ldcg(&args.part_ml[(sbase_p + sp) * r + h]).x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float l = 0.f;
-    for (int sp = lane; sp < args.splits; sp += 32) {
+    for (int sp = lane; sp < S; sp += 32) {
       const float2 ml = __ldcg(&args.part_ml[(sbase_p + sp) * r + h]);
       l += (ml.x == -INFINITY) ? 0.f : ml.y * ex2_approx(ml.x - M);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    for (int d = lane; d < D; d += 32) {
-      float acc = 0.f;
-      for (int sp = 0; sp < args.splits; ++sp) {
-        const float mx = __ldcg(&args.part_ml[(sbase_p + sp) * r + h]).x;
-        const float wt = (mx == -INFINITY) ? 0.f : ex2_approx(mx - M);
-        acc += wt * __ldcg(&args.part_o[((sbase_p + sp) * r + h) * D + d]);
-      }
-      args.o[((size_t)b * args.Hq + g * r + h) * D + d] = __float2bfloat16_rn(acc * inv);
+    for (int sp = lane; sp < S; sp += 32) {
+      const float mx = __ldcg(&args.part_ml[(sbase_p + sp) * r + h]).x;
+      wts[h * S + sp] = (mx == -INFINITY) ? 0.f : ex2_approx(mx - M) * inv;
     }
     if (lane == 0 && args.lse != nullptr)
       args.lse[(size_t)b * args.Hq + g * r + h] = (M + __log2f(l)) * 0.69314718055994531f;
+  }
+  named_sync_consumers();
+  for (int idx = threadIdx.x; idx < r * D; idx += kCons) {
+    const int h = idx / D, d = idx % D;
+    const float* po = args.part_o + (sbase_p * r + h) * D + d;  // split sp at + sp * r * D
+    float acc = 0.f;
+#pragma unroll 8
+    for (int sp = 0; sp < S; ++sp) acc += wts[h * S + sp] * __ldcg(po + (size_t)sp * r * D);
+    args.o[((size_t)b * args.Hq + g * r + h) * D + d] = __float2bfloat16_rn(acc);
   }
   if (threadIdx.x == 0) args.counters[b * args.Hkv + g] = 0;  // ready for the next call
 }

@@ -86,7 +86,7 @@ int decode_splits_max(int B, int Hkv) {
   const int slots = 2 * device_sms();
   int s = (2 * slots + B * Hkv - 1) / (B * Hkv);
   if (s < 1) s = 1;
-  if (s > 4096) s = 4096;
+  if (s > 2048) s = 2048;  // the final merge keeps r x splits weights in shared memory
   return s;
 }
 
