@@ -200,6 +200,20 @@ def gen_on_device(shape, seed, dev):
 # our arm
 # ---------------------------------------------------------------------------
 
+def bench_config(world):
+    """The workload description both arms print (the reference arm times the
+    oracle on the prefill part of it)."""
+    P, Dc = PREFILL, DECODE
+    return {
+        "workload": P["workload"] + " + " + Dc["workload"],
+        "prefill": {k_: P[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")},
+        "decode": {k_: Dc[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")},
+        "query_shift": "self_extend",
+        "l2": "inputs larger than L2",
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+    }
+
+
 def run_ours(args):
     import torch
     from rope_context_extension_b200 import jetlong as jl
@@ -457,7 +471,8 @@ def run_ours(args):
     traffic = load_traffic() if not (args.prefill_len or args.decode_len or args.decode_batch) else {}
     out = None
     if rank == 0:
-        cpu = None if args.no_cpu_baseline else cpu_baseline_sample(seconds=args.cpu_seconds)
+        # the oracle's CPU baseline is taken on rank 0 of a one-GPU run only
+        cpu = None if (args.no_cpu_baseline or world > 1) else cpu_baseline_sample(seconds=args.cpu_seconds)
         out = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -471,14 +486,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded randn on device, N(0,1) bf16; inputs larger than L2, no flush)",
-            "config": {
-                "workload": P["workload"] + " + " + Dc["workload"],
-                "prefill": {k_: P[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")},
-                "decode": {k_: Dc[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")},
-                "query_shift": "self_extend",
-                "l2": "inputs larger than L2",
-                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            },
+            "config": bench_config(world),
             "prefill": {"ms": round(pre_ms_max, 3), "correction_ms": round(corr_ms, 3),
                         "attention_ms": round(attn_ms_max, 3), "tokens_per_s": round(world * P["L"] * P["B"] /
                                                                                      (pre_ms_max * 1e-3), 1),
@@ -600,8 +608,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded randn, N(0,1) bf16 widened to fp64)",
-        "config": {"workload": PREFILL["workload"],
-                   "prefill": {k_: PREFILL[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")}},
+        "config": bench_config(1),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
                          "sample": f"each step: {args.ref_rows} random query rows x 4 q heads of one KV head of "
                                    f"the 128K prefill workload on the fp64 CPU oracle"},
