@@ -79,8 +79,8 @@ enum {
   kVFull = kKEmpty + kStages,
   kVEmpty = kVFull + kStages,
   kSFull = kVEmpty + kStages,  // 2
-  kPFull = kSFull + 2,         // 2
-  kOFinal = kPFull + 2,
+  kPFull = kSFull + 2,         // 4: [head][64-key half of P]
+  kOFinal = kPFull + 4,
   kDrain = kOFinal + 1,
   kNumBars = kDrain + 1
 };
@@ -201,7 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(bar(kSFull + h), 1);
-      mbar_init(bar(kPFull + h), 128);
+      mbar_init(bar(kPFull + 2 * h), 128);
+      mbar_init(bar(kPFull + 2 * h + 1), 128);
     }
     mbar_init(bar(kOFinal), 1);
     mbar_init(bar(kDrain), 1);
@@ -355,20 +356,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return true;
       };
+      // O_h += P V in two 64-key halves, each issued as soon as the softmax
+      // has written that half of P, so the first half's product runs while
+      // the second half's exponentials are taken.
       auto issue_pv = [&](int h, int p) -> bool {
         const int s = p % C::kVStages;
         const uint32_t ph = (uint32_t)(p / C::kVStages) & 1u;
         if (h == 0 && !mbar_wait(bar(kVFull + s), ph, abort_flag, args.dev_error)) return false;
-        if (!mbar_wait(bar(kPFull + h), (uint32_t)p & 1u, abort_flag, args.dev_error)) return false;
-        tc_fence_after();
         const uint32_t va = sbase + C::kVOff + s * C::kTileBytes;
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks) {
-          // V tile is MN-major for this product: 64-dim slabs kChunkBytes apart
-          // (leading offset), 8-key groups 1024 B apart (stride offset).
-          mma_ts(tmem + o_col(h), tmem + s_col(h) + (uint32_t)(ks * 8),
-                 make_sdesc_sw128(va + (uint32_t)(ks * 2048), kChunkBytes, 1024), id_pv,
-                 (p > 0 || ks > 0) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(bar(kPFull + 2 * h + half), (uint32_t)p & 1u, abort_flag, args.dev_error)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBN / 32; ++kk) {
+            const int ks = half * (kBN / 32) + kk;
+            // V tile is MN-major for this product: 64-dim slabs kChunkBytes apart
+            // (leading offset), 8-key groups 1024 B apart (stride offset).
+            mma_ts(tmem + o_col(h), tmem + s_col(h) + (uint32_t)(ks * 8),
+                   make_sdesc_sw128(va + (uint32_t)(ks * 2048), kChunkBytes, 1024), id_pv,
+                   (p > 0 || ks > 0) ? 1u : 0u);
+          }
         }
         if (h == NH - 1) tc_commit(bar(kVEmpty + s));
         return true;
@@ -471,8 +479,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
 
+      // O_h must be rescaled before either half of this pass's P V; in the
+      // (rare) passes that need it, both halves of P are released after it.
+      const bool resc = __any_sync(0xffffffffu, rescale_o) && p > 0;
       // p = 2^(s * scale * log2 e - m): one packed FMA per pair, the row sum in
-      // two packed accumulators.
+      // two packed accumulators; otherwise each 64-key half of P is released to
+      // the MMA warp as soon as it is in TMEM.
       const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-msub, -msub);
       uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
@@ -494,28 +506,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[k] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_addr + half * 32, pk);
+        if (half == 0 && resc) continue;
+        if (half == 1 && resc) {
+          // O_h(p-1) is final here: its product was issued before S_h(p).
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(o_addr + c * 32, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+            tmem_st32(o_addr + c * 32, ov);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        if (half == 1 && resc) mbar_arrive(bar(kPFull + 2 * h));
+        mbar_arrive(bar(kPFull + 2 * h + half));
       }
       {
         float a0, a1;
         f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
         l_sum += a0 + a1;
       }
-
-      if (__any_sync(0xffffffffu, rescale_o) && p > 0) {
-        // O_h(p-1) is final here: its product was issued before S_h(p).
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(o_addr + c * 32, ov);
-          tmem_ld_wait(ov);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-          tmem_st32(o_addr + c * 32, ov);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(kPFull + h));
     }
 
     if (ok) {
