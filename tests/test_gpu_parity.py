@@ -97,7 +97,7 @@ def test_prefill_full_size_sampled(name, B, L, Hq, Hkv, W, w0):
     q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, 128, seed=0)
     o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6)
     assert err == 0
-    rows = sample_rows(L, w0, 40, seed=1)
+    rows = sample_rows(L, w0, 256, seed=1)  # >= 256 rows per head, band and tile edges included
     heads = sorted({0, 1, Hq // 2 + 1, Hq - 1})
     p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
     ref = oracle_prefill_rows(q, k, v, rows, heads, p)
@@ -212,7 +212,7 @@ def test_prefill_split_mode_full_size_sampled():
     q, k, v = synthetic.prefill_inputs(1, L, 32, 8, 128, seed=0)
     o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6, split=True)
     assert err == 0
-    rows = sample_rows(L, w0, 24, seed=2)
+    rows = sample_rows(L, w0, 256, seed=2)
     heads = [0, 17, 31]
     p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
     ref = oracle_prefill_rows(q, k, v, rows, heads, p)
