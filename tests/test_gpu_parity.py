@@ -51,6 +51,7 @@ CASES = [
     (1, 129, 2, 1, 64, 50, 128, jo.MODE_SELF_EXTEND, 0.0),      # one row past a tile
     (1, 1, 2, 1, 128, 16, 0, jo.MODE_SELF_EXTEND, 0.0),         # single token
     (1, 1300, 8, 2, 128, 260, 1, jo.MODE_SELF_EXTEND, 0.01),    # w0 = 1: only the diagonal is local
+    (3, 700, 16, 2, 128, 200, 150, jo.MODE_SELF_EXTEND, 0.0),   # GQA 8 (4 CTAs per KV head and block), B 3
 ]
 
 
