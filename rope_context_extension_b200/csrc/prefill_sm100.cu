@@ -43,10 +43,10 @@ constexpr int kLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 
 constexpr int kLowRegs = 104;     // warpgroup 0: TMA producer, MMA issuer
 constexpr int kHighRegs = 200;    // warpgroups 1-2: softmax
 // kPolyEvery > 0 sends one pair of exponentials in every kPolyEvery to the FMA
-// pipe (ex2_poly2) instead of the MUFU.  Measured at the 128K workload with
-// one pair in four: 879 TFLOP/s against 1000-1040 with all exponentials on the
-// MUFU — the softmax is bound by issue and latency, not by MUFU throughput —
-// so it is off.
+// pipe (ex2_poly2, which uses no MUFU or conversion instruction) instead of the
+// MUFU.  Measured at the 128K workload: one pair in four 1026-1030 TFLOP/s and
+// one in eight 1006-1016, against 1031 with every exponential on the MUFU.  The
+// softmax is bound by latency, not by MUFU throughput, so it is off.
 constexpr int kPolyEvery = 0;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kChunkBytes = 128 * 128;  // one 128-row x 128-byte swizzled slab
