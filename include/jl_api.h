@@ -281,11 +281,25 @@ int jl_decode_combine(const void* o_parts, const float* lse_parts, int parts, vo
 
 /*
  * Diagnostic: evaluates, on the device, the FMA-pipe exponential that the
- * prefill softmax uses for part of each row (Cody-Waite reduction plus a fitted
- * degree-3 polynomial) and CUDA's exp2f on the same n inputs (device arrays),
- * so its error can be checked.  Not part of the attention path.
+ * prefill softmax can use for part of each row (Cody-Waite reduction plus a
+ * fitted degree-3 polynomial; off by default) and CUDA's exp2f on the same n
+ * inputs (device arrays), so its error can be checked.  Not part of the
+ * attention path.
  */
 int jl_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, void* stream);
+
+/*
+ * Self-test of the failure path every pipeline wait shares (no counterpart on
+ * the pages): one tiny kernel waits, with the same bounded mbarrier wait, on a
+ * barrier that nothing completes.  After timeout_s seconds (0 < timeout_s <= 10)
+ * that wait gives up and writes 1 (the device-timeout code) to *dev_error (a
+ * device int); a second warp waiting on another such barrier gives up as soon
+ * as the first has aborted.  A wait that returned success would write 99.  The
+ * kernel then returns normally, so the context stays usable.  Asynchronous on
+ * `stream`; read *dev_error after synchronising.
+ * Errors: JL_ERR_INVALID_ARG (null dev_error, timeout out of range), JL_ERR_CUDA.
+ */
+int jl_wait_timeout_check(int* dev_error, double timeout_s, void* stream);
 
 /*
  * jl_bifocal_decode without a workspace argument, for callers that cannot

@@ -95,7 +95,32 @@ __global__ void exp2_poly_check_kernel(const float* x, float* y_poly, float* y_r
   }
 }
 
+// Exercises the pipelines' bounded wait on a barrier that nothing completes:
+// warp 0 waits until its limit runs out (it must return false and write the
+// timeout code), warp 1 waits on a second such barrier and must give up as soon
+// as warp 0 has aborted.  A wait that returned true writes 99 instead.
+__global__ void wait_timeout_check_kernel(int* dev_error, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bars[0]), 1);
+    mbar_init(smem_addr(&bars[1]), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int w = threadIdx.x >> 5;
+  const bool ok = mbar_wait(smem_addr(&bars[w]), 0u, &abort_flag, w == 0 ? dev_error : nullptr,
+                            w == 0 ? timeout_ns : 4 * timeout_ns);
+  if (ok && (threadIdx.x & 31) == 0) atomicExch(dev_error, 99);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_check(int* dev_error, unsigned long long timeout_ns, cudaStream_t stream) {
+  wait_timeout_check_kernel<<<1, 64, 0, stream>>>(dev_error, timeout_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream) {
   const int pairs = (n + 1) / 2;

@@ -551,6 +551,14 @@ int jl_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, void*
   return JL_OK;
 }
 
+int jl_wait_timeout_check(int* dev_error, double timeout_s, void* stream) {
+  if (!dev_error || !(timeout_s > 0.0) || timeout_s > 10.0) return JL_ERR_INVALID_ARG;
+  if (jl::launch_wait_timeout_check(dev_error, (unsigned long long)(timeout_s * 1e9),
+                                    reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
+}
+
 int jl_rope_append(const void* q_raw, const void* k_raw, const void* v_new, const int32_t* positions, void* q_out,
                    void* k_cache, void* v_cache, int64_t cache_len, int B, int Hq, int Hkv, int head_dim,
                    double rope_base, int* dev_error, void* stream) {

@@ -66,16 +66,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity.  Returns false (and makes
 // every other waiter of the CTA give up too, through *abort) once the wait has
-// run for kWaitTimeoutNs, or as soon as another thread has aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* dev_error) {
+// run for timeout_ns (kWaitTimeoutNs in every pipeline), or as soon as another
+// thread has aborted; the first to run out writes kDevTimeout to *dev_error.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* dev_error,
+                                          uint64_t timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0u) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
         if (dev_error) atomicExch(dev_error, kDevTimeout);
         return false;

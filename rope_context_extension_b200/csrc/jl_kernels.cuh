@@ -92,6 +92,7 @@ struct CombineArgs {
 };
 cudaError_t launch_lse_combine(const CombineArgs& a, int D, cudaStream_t stream);
 cudaError_t launch_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream);
+cudaError_t launch_wait_timeout_check(int* dev_error, unsigned long long timeout_ns, cudaStream_t stream);
 
 // Base RoPE of one new token per sequence and its append to the KV cache.
 struct AppendArgs {

@@ -19,7 +19,7 @@ __all__ = [
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
     "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes", "jl_bifocal_prefill_ie", "jl_bifocal_decode_range",
-    "jl_decode_combine", "jl_exp2_poly_check", "EXPORTED_SYMBOLS",
+    "jl_decode_combine", "jl_exp2_poly_check", "jl_wait_timeout_check", "EXPORTED_SYMBOLS",
 ]
 
 JL_QSHIFT_NONE = 0
@@ -31,6 +31,7 @@ EXPORTED_SYMBOLS = (
     "jl_prefill_attention", "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append",
     "jl_prefill_chunk_workspace_bytes", "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes",
     "jl_bifocal_prefill_ie", "jl_bifocal_decode_range", "jl_decode_combine", "jl_exp2_poly_check",
+    "jl_wait_timeout_check",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -99,6 +100,8 @@ def lib() -> ctypes.CDLL:
     L.jl_decode_combine.restype = c_i
     L.jl_exp2_poly_check.argtypes = [c_p, c_p, c_p, c_i, c_p]
     L.jl_exp2_poly_check.restype = c_i
+    L.jl_wait_timeout_check.argtypes = [c_p, c_d, c_p]
+    L.jl_wait_timeout_check.restype = c_i
     _lib = L
     return L
 
@@ -392,3 +395,11 @@ def jl_exp2_poly_check(x):
     yr = torch.empty_like(x)
     _check(lib().jl_exp2_poly_check(_ptr(x), _ptr(yp), _ptr(yr), x.numel(), _stream(None)), "jl_exp2_poly_check")
     return yp, yr
+
+
+def jl_wait_timeout_check(dev_error, timeout_s: float = 0.2, stream=None):
+    """Launch the bounded-wait self-test; dev_error is a device int32 tensor
+    (read it after synchronising: 1 = the wait ran out as it should)."""
+    import torch
+    _check_tensor(dev_error, "dev_error", torch.int32)
+    _check(lib().jl_wait_timeout_check(_ptr(dev_error), float(timeout_s), _stream(stream)), "jl_wait_timeout_check")

@@ -155,3 +155,10 @@ def test_prefill_chunk_argument_errors(lib):
     assert chunk(ws_bytes=need - 1) == JL_ERR_WORKSPACE
     # a whole-sequence chunk needs what jl_prefill_workspace_bytes reports
     assert lib.jl_prefill_chunk_workspace_bytes(2, 0, 300, 8, 2, 64) == lib.jl_prefill_workspace_bytes(2, 300, 8, 2, 64)
+
+
+def test_wait_timeout_check_argument_errors(lib):
+    # rejected before any launch (no GPU needed)
+    assert lib.jl_wait_timeout_check(None, 0.1, None) == JL_ERR_INVALID_ARG
+    assert lib.jl_wait_timeout_check(A, 0.0, None) == JL_ERR_INVALID_ARG
+    assert lib.jl_wait_timeout_check(A, 11.0, None) == JL_ERR_INVALID_ARG
