@@ -121,6 +121,18 @@ def test_prefill_argument_errors(lib):
     assert _prefill(lib, ws=A + 4) == JL_ERR_ALIGNMENT
 
 
+def test_empty_inputs_are_rejected_before_any_launch(lib):
+    # no batch, no head, no token: every entry point refuses, nothing launches
+    assert _prefill(lib, B=0) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, Hq=0) == JL_ERR_INVALID_ARG
+    assert _prefill(lib, Hkv=0) == JL_ERR_INVALID_ARG
+    assert _decode(lib, B=0) == JL_ERR_INVALID_ARG
+    assert _decode(lib, L=0) == JL_ERR_INVALID_ARG
+    assert _decode(lib, Hq=0) == JL_ERR_INVALID_ARG
+    assert lib.jl_decode_workspace_bytes(1, 0, 4, 2, 128) == 0
+    assert lib.jl_prefill_workspace_bytes(1, 0, 4, 2, 128) == 0
+
+
 def test_decode_argument_errors(lib):
     assert _decode(lib, D=80) == JL_ERR_UNSUPPORTED
     assert _decode(lib, Hq=32, Hkv=2) == JL_ERR_UNSUPPORTED  # more than 8 query heads per KV head
