@@ -92,6 +92,21 @@ int jl_remote_positions(int64_t L, int64_t w0, int64_t w_pretrained, int mode, i
                         int32_t* k_pos_out);
 
 /*
+ * Tile schedule of jl_bifocal_prefill over a whole sequence of length L, per
+ * (batch, query head), from the same functions the attention kernel runs.
+ * A causal pair (i, j) is local when i - j < w0 and remote otherwise (Jet-Long
+ * review, "Method"); a 128 x 128 tile holding both kinds gets a local and a
+ * remote pass with complementary masks.  When G = 1 or w0 >= L every tile gets
+ * one local pass (the method is then exactly base RoPE).  Host only.
+ * counts_out[4] (caller-owned): [0] tiles with a local pass only, [1] tiles
+ * with both passes, [2] tiles with a remote pass only, [3] passes in total
+ * ([0] + 2 [1] + [2]).
+ * Errors: JL_ERR_INVALID_ARG for a NULL counts_out, L < 1 or L > 2^30, w0 < 0
+ * or w_pretrained < 1.
+ */
+int jl_prefill_tile_classes(int64_t L, int64_t w0, int64_t w_pretrained, int64_t* counts_out);
+
+/*
  * Scratch bytes jl_bifocal_prefill needs: space for the remote-rotated Q and K
  * rows (2 * B * L * (Hq + Hkv) * D bytes plus alignment); twice this with
  * JL_REMOTE_SPLIT in `mode`.  0 on bad arguments.

@@ -125,6 +125,46 @@ def remote_relative_range(L: int, w0: int, w_pretrained: int, mode: str):
     return lo, hi
 
 
+def tile_classes(L: int, w0: int, tile: int = 128, exhaustive: bool = False):
+    """Counts of the causal tile x tile blocks of an L x L score matrix by the
+    pair classes they hold: (local only, both, remote only).
+
+    From the definitions alone: a causal pair (i, j), j <= i < L, is local iff
+    ``is_local`` (i - j < w0), remote otherwise (Jet-Long review, "Method").
+    Block (a, c), c <= a, holds query rows tile*a .. and keys tile*c ..; it
+    holds a causal pair whenever c <= a.  ``exhaustive`` enumerates every pair
+    of every block (small L); otherwise the causal distances i - j of a block,
+    a contiguous integer range, are bounded by their ends: the smallest is
+    max(0, tile*(a - c) - (tile - 1)) and the largest
+    min(tile*a + tile - 1, L - 1) - tile*c.
+    """
+    if L < 1 or w0 < 0 or tile < 1:
+        raise ValueError("need L >= 1, w0 >= 0, tile >= 1")
+    nb = -(-L // tile)
+    loc_only = both = rem_only = 0
+    for a in range(nb):
+        i = np.arange(tile * a, min(tile * a + tile, L), dtype=np.int64)
+        for c in range(a + 1):
+            if exhaustive:
+                j = np.arange(tile * c, min(tile * c + tile, L), dtype=np.int64)
+                dist = i[:, None] - j[None, :]
+                causal = dist >= 0
+                has_loc = bool(np.any(causal & (dist < w0)))
+                has_rem = bool(np.any(causal & (dist >= w0)))
+            else:
+                dmin = max(0, tile * (a - c) - (tile - 1))
+                dmax = int(i[-1]) - tile * c
+                has_loc = dmin < w0
+                has_rem = dmax >= w0
+            if has_loc and has_rem:
+                both += 1
+            elif has_loc:
+                loc_only += 1
+            elif has_rem:
+                rem_only += 1
+    return loc_only, both, rem_only
+
+
 # ---------------------------------------------------------------------------
 # RoPE (half-split pairs), fp64
 # ---------------------------------------------------------------------------

@@ -163,6 +163,36 @@ int jl_remote_positions(int64_t L, int64_t w0, int64_t w_pretrained, int mode, i
   return JL_OK;
 }
 
+int jl_prefill_tile_classes(int64_t L, int64_t w0, int64_t w_pretrained, int64_t* counts_out) {
+  if (counts_out == nullptr || L < 1 || L > (int64_t(1) << 30) || w0 < 0 || w_pretrained < 1)
+    return JL_ERR_INVALID_ARG;
+  const int64_t G = jl::group_size(L, w_pretrained);
+  const bool al = jl::all_local(L, w0, G);
+  // the band width the attention launch hands the kernel
+  const int w0k = al ? (1 << 30) : (int)w0;
+  int64_t loc_only = 0, both = 0, rem_only = 0, passes = 0;
+  for (int mb = 0; mb < (int)((L + 127) / 128); ++mb) {
+    const int last = (int)std::min<int64_t>(mb * 128 + 127, L - 1);
+    const jl::Sched s = jl::make_sched<jl::kBifocal>(mb * 128, last, w0k, al);
+    // local passes visit blocks nb_max - n_loc + 1 .. nb_max, remote passes 0 .. nb_rem_max
+    int ov = 0;
+    if (s.n_loc > 0 && s.n_rem > 0) {
+      const int lo = s.nb_max - s.n_loc + 1;
+      const int hi = s.nb_rem_max < s.nb_max ? s.nb_rem_max : s.nb_max;
+      ov = hi >= lo ? hi - lo + 1 : 0;
+    }
+    both += ov;
+    loc_only += s.n_loc - ov;
+    rem_only += s.n_rem - ov;
+    passes += s.n_loc + s.n_rem;
+  }
+  counts_out[0] = loc_only;
+  counts_out[1] = both;
+  counts_out[2] = rem_only;
+  counts_out[3] = passes;
+  return JL_OK;
+}
+
 size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
   return round_up((size_t)B * L * Hq * head_dim * 2) + round_up((size_t)B * L * Hkv * head_dim * 2);

@@ -2,6 +2,7 @@
 #pragma once
 
 #include "jl_common.cuh"
+#include "jl_sched.h"
 
 namespace jl {
 
@@ -38,7 +39,6 @@ struct PrefillArgs {
   int kind;          // kBifocal, or one call of the inclusion-exclusion formulation
   float scale_log2;  // softmax scale * log2(e)
 };
-enum : int { kBifocal = 0, kWindowBase = 1, kCausalRemote = 2, kWindowRemote = 3 };
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
                            const CUtensorMap& tm_kr_lo, const PrefillArgs& a, int D, bool split,

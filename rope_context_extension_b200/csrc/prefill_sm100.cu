@@ -86,65 +86,6 @@ enum {
 };
 static_assert(kNumBars * 8 <= 192, "barrier block overflow");
 
-// Pass schedule of one query block whose first query position is `off`
-// (query rows off .. off + 127; keys in 128-key blocks nb).  Block nb spans
-// i - j in [off - 128 nb - 127, off - 128 nb + 127].  Local passes run on the
-// key blocks nb_max, nb_max - 1, ... that hold a pair with 0 <= i - j < w0;
-// remote passes on nb_rem_max, ..., 0 (the blocks with a pair i - j >= w0).
-struct Sched {
-  int n_loc, n_rem, nb_max, nb_rem_max;
-};
-
-__device__ __forceinline__ int floor_div128(int x) { return x >= 0 ? x / 128 : -((127 - x) / 128); }
-
-// kind: kBifocal (local passes, then remote passes: the fused method), or one
-// of the three calls of the inclusion-exclusion formulation (Jet-Long review,
-// "Method"): kWindowBase (A: pairs with 0 <= i - j < w0, base rows),
-// kCausalRemote (B: every causal pair, corrected rows), kWindowRemote (C: the
-// window of A, corrected rows).
-template <int kind>
-__device__ __forceinline__ Sched make_sched(int off, int w0, bool all_local) {
-  Sched s;
-  s.nb_max = (off + 127) / 128;  // last block holding a causal key
-  if (kind == kCausalRemote) {
-    s.n_loc = 0;
-    s.nb_rem_max = s.nb_max;
-    s.n_rem = s.nb_max + 1;
-    return s;
-  }
-  if (all_local) {
-    s.n_loc = s.nb_max + 1;
-    s.n_rem = 0;
-    s.nb_rem_max = -1;
-    return s;
-  }
-  if (w0 > 0) {
-    const int nb_loc_min = max(0, floor_div128(off - 127 - w0) + 1);  // 128 nb > off - 127 - w0
-    s.n_loc = max(0, s.nb_max - nb_loc_min + 1);
-  } else {
-    s.n_loc = 0;
-  }
-  s.nb_rem_max = floor_div128(off + 127 - w0);  // 128 nb <= off + 127 - w0
-  s.n_rem = kind == kBifocal ? max(0, s.nb_rem_max + 1) : 0;
-  return s;
-}
-
-__device__ __forceinline__ int pass_block(const Sched& s, int p) {
-  return p < s.n_loc ? s.nb_max - p : s.nb_rem_max - (p - s.n_loc);
-}
-// Does pass p read the corrected (remote-position) Q / K rows?
-template <int kind>
-__device__ __forceinline__ bool pass_remote_ops(const Sched& s, int p) {
-  return kind == kBifocal ? p >= s.n_loc : (kind != kWindowBase);
-}
-// Which pairs of the tile pass p keeps: 0 band (0 <= i-j < w0), 1 beyond the
-// band (i-j >= w0), 2 every causal pair (i-j >= 0).
-template <int kind>
-__device__ __forceinline__ int pass_mask_kind(const Sched& s, int p) {
-  if (kind == kCausalRemote) return 2;
-  return p < s.n_loc ? 0 : 1;
-}
-
 __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
   // Used only after an abort: wait (up to ~100 ms) for async work already in
   // flight so the CTA never exits while a copy or an MMA still targets it.
@@ -219,7 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
   const int off = args.q_off + mb * kBM;  // position of this block's first query
-  const Sched sc = make_sched<kKind>(off, args.w0, args.all_local != 0);
+  const int last = min(off + kBM - 1, args.q_off + args.Lq - 1);  // last query row of the block
+  const Sched sc = make_sched<kKind>(off, last, args.w0, args.all_local != 0);
   const int npass = sc.n_loc + sc.n_rem;
   const bool q_switch = sc.n_loc > 0 && sc.n_rem > 0;
   const int w0 = args.w0;

@@ -19,7 +19,8 @@ __all__ = [
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
     "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes", "jl_bifocal_prefill_ie", "jl_bifocal_decode_range",
-    "jl_decode_combine", "jl_exp2_poly_check", "jl_wait_timeout_check", "EXPORTED_SYMBOLS",
+    "jl_decode_combine", "jl_exp2_poly_check", "jl_wait_timeout_check", "jl_prefill_tile_classes",
+    "EXPORTED_SYMBOLS",
 ]
 
 JL_QSHIFT_NONE = 0
@@ -31,7 +32,7 @@ EXPORTED_SYMBOLS = (
     "jl_prefill_attention", "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append",
     "jl_prefill_chunk_workspace_bytes", "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes",
     "jl_bifocal_prefill_ie", "jl_bifocal_decode_range", "jl_decode_combine", "jl_exp2_poly_check",
-    "jl_wait_timeout_check",
+    "jl_wait_timeout_check", "jl_prefill_tile_classes",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -61,6 +62,8 @@ def lib() -> ctypes.CDLL:
     L.jl_group_size.restype = c_i
     L.jl_remote_positions.argtypes = [c_i64, c_i64, c_i64, c_i, c_p, c_p]
     L.jl_remote_positions.restype = c_i
+    L.jl_prefill_tile_classes.argtypes = [c_i64, c_i64, c_i64, c_p]
+    L.jl_prefill_tile_classes.restype = c_i
     L.jl_prefill_workspace_bytes.argtypes = [c_i, c_i, c_i, c_i, c_i]
     L.jl_prefill_workspace_bytes.restype = c_sz
     L.jl_decode_workspace_bytes.argtypes = [c_i, c_i, c_i, c_i, c_i]
@@ -135,6 +138,14 @@ def jl_remote_positions(L: int, w0: int, w_pretrained: int, mode: int = JL_QSHIF
     _check(lib().jl_remote_positions(L, w0, w_pretrained, mode, q.ctypes.data, k.ctypes.data),
            "jl_remote_positions")
     return q, k
+
+
+def jl_prefill_tile_classes(L: int, w0: int, w_pretrained: int):
+    """(local-only tiles, tiles with both passes, remote-only tiles, passes) of the
+    prefill's 128 x 128 tile schedule over a length-L sequence (host call)."""
+    out = np.zeros(4, dtype=np.int64)
+    _check(lib().jl_prefill_tile_classes(L, w0, w_pretrained, out.ctypes.data), "jl_prefill_tile_classes")
+    return tuple(int(x) for x in out)
 
 
 def jl_prefill_workspace_bytes(B: int, L: int, Hq: int, Hkv: int, head_dim: int) -> int:

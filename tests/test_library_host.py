@@ -72,6 +72,39 @@ def test_remote_positions_bit_exact(lib, L, w0, W, mode):
     np.testing.assert_array_equal(k, fk.astype(np.int32))
 
 
+TILE_CASES = [(L, w0) for L in (1, 127, 128, 129, 200, 383, 640, 777, 1000, 1300, 2049)
+              for w0 in (0, 1, 31, 127, 128, 129, 300, 1000, 5000)]
+
+
+@pytest.mark.parametrize("L,w0", TILE_CASES)
+def test_prefill_tile_schedule_matches_pair_classes(lib, L, w0):
+    # The attention kernel's tile schedule (local pass, remote pass or both per
+    # 128 x 128 block) against the oracle's classification of the blocks' pairs.
+    W = max(1, L // 3)
+    loc, both, rem, passes = jl.jl_prefill_tile_classes(L, w0, W)
+    assert passes == loc + 2 * both + rem
+    if jo.group_size(L, W) == 1 or w0 >= L:
+        nb = -(-L // 128)
+        assert (loc, both, rem) == (nb * (nb + 1) // 2, 0, 0)  # exactly base RoPE: one local pass per block
+    else:
+        assert (loc, both, rem) == jo.tile_classes(L, w0)
+
+
+@pytest.mark.parametrize("L,w0,W", [(131072, 4096, 32768), (65536, 4096, 32768), (512, 32, 128), (100003, 4096, 32768),
+                                    (131072, 0, 32768)])
+def test_prefill_tile_schedule_full_workloads(lib, L, w0, W):
+    assert jl.jl_prefill_tile_classes(L, w0, W)[:3] == jo.tile_classes(L, w0)
+
+
+def test_prefill_tile_classes_rejects_bad_args(lib):
+    out = (ctypes.c_int64 * 4)()
+    assert lib.jl_prefill_tile_classes(0, 0, 10, out) == JL_ERR_INVALID_ARG
+    assert lib.jl_prefill_tile_classes(10, -1, 10, out) == JL_ERR_INVALID_ARG
+    assert lib.jl_prefill_tile_classes(10, 0, 0, out) == JL_ERR_INVALID_ARG
+    assert lib.jl_prefill_tile_classes(10, 0, 10, None) == JL_ERR_INVALID_ARG
+    assert lib.jl_prefill_tile_classes((1 << 30) + 1, 0, 10, out) == JL_ERR_INVALID_ARG
+
+
 def test_remote_positions_rejects_bad_args(lib):
     assert lib.jl_remote_positions(0, 0, 10, 1, None, None) == JL_ERR_INVALID_ARG
     assert lib.jl_remote_positions(10, -1, 10, 1, None, None) == JL_ERR_INVALID_ARG

@@ -92,6 +92,29 @@ def test_rope_d2_is_plane_rotation():
         np.testing.assert_allclose(jo.rope_rotate(x, p, 10000.0), want, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("L,w0", [(1, 0), (5, 3), (128, 0), (129, 1), (200, 100), (300, 129), (512, 32),
+                                  (640, 256), (777, 300), (1000, 1), (1024, 5000)])
+def test_tile_classes_closed_form_equals_pair_enumeration(L, w0):
+    # brute force over every pair of every 128 x 128 block
+    assert jo.tile_classes(L, w0) == jo.tile_classes(L, w0, exhaustive=True)
+
+
+def test_tile_classes_by_hand():
+    # L 512, w0 32: four diagonal blocks hold distances 0..127 and the three
+    # first sub-diagonal blocks 1..255, so all seven straddle the band edge;
+    # the three blocks two or more apart hold distances >= 129: remote only.
+    assert jo.tile_classes(512, 32) == (0, 7, 3)
+    # w0 0: no local pair; w0 >= L: no remote pair (10 causal blocks at L 512)
+    assert jo.tile_classes(512, 0) == (0, 0, 10)
+    assert jo.tile_classes(512, 512) == (10, 0, 0)
+    # w0 1: only i == j is local, so only the four diagonal blocks hold it
+    assert jo.tile_classes(512, 1) == (0, 4, 6)
+    # tile 1: every pair is its own block
+    L, w0 = 9, 3
+    n_loc = sum(1 for i in range(L) for j in range(i + 1) if i - j < w0)
+    assert jo.tile_classes(L, w0, tile=1) == (n_loc, 0, L * (L + 1) // 2 - n_loc)
+
+
 def test_rope_frequencies_closed_form():
     th = jo.rope_frequencies(8, 10000.0)
     np.testing.assert_allclose(th, [1.0, 0.1, 0.01, 0.001], rtol=1e-14)
