@@ -369,38 +369,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mkind = pass_mask_kind<kKind>(sc, p);
       const int dd0 = off - 128 * pass_block(sc, p);  // i - j at row 0, column 0
 
+      // S in two 64-column halves: the first half's mask and partial row max
+      // run while the second half's load is in flight (tcgen05.wait::ld
+      // waits for every outstanding load, so the second pair is issued after
+      // the first wait).
       uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+      tmem_ld32(s_addr, sr[0]);
+      tmem_ld32(s_addr + 32, sr[1]);
+      tmem_ld_wait(sr[0]);
+      tmem_ld_wait(sr[1]);
+      tmem_ld32(s_addr + 64, sr[2]);
+      tmem_ld32(s_addr + 96, sr[3]);
 
       float x[128];  // raw scores (fp32 accumulator values)
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]);
-
       const bool need_mask = mkind == 1 ? (dd0 - 127 < w0)
                              : mkind == 0 ? (dd0 - 127 < 0 || dd0 + 127 >= w0)
                                           : (dd0 - 127 < 0);
-      if (need_mask) {
-        const int dd = dd0 + row;  // i - j = dd - col
+      const int dd = dd0 + row;  // i - j = dd - col
+      float m4[4];
+      auto take = [&](int c0) {
 #pragma unroll
-        for (int col = 0; col < 128; ++col) {
-          const int rel = dd - col;
-          const bool keep = mkind == 1 ? (rel >= w0) : mkind == 0 ? (rel >= 0 && rel < w0) : (rel >= 0);
-          if (!keep) x[col] = -INFINITY;
+        for (int c = c0; c < c0 + 2; ++c)
+#pragma unroll
+          for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]);
+        if (need_mask) {
+#pragma unroll
+          for (int col = c0 * 32; col < c0 * 32 + 64; ++col) {
+            const int rel = dd - col;
+            const bool keep = mkind == 1 ? (rel >= w0) : mkind == 0 ? (rel >= 0 && rel < w0) : (rel >= 0);
+            if (!keep) x[col] = -INFINITY;
+          }
         }
-      }
+      };
       // Row max over four independent chains of three-input maxima (the scale
       // is positive, so the max of the raw scores scales to the max of the
       // scaled ones).
-      float m4[4];
+      take(0);
 #pragma unroll
       for (int j = 0; j < 4; ++j) m4[j] = fmaxf(x[j], x[4 + j]);
 #pragma unroll
-      for (int col = 8; col < 128; col += 8)
+      for (int col = 8; col < 64; col += 8)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m4[j] = fmax3(m4[j], x[col + j], x[col + 4 + j]);
+      // (the partial maxima are tied to this wait, so they are taken while the
+      // second half of S is in flight)
+      asm volatile("tcgen05.wait::ld.sync.aligned;" : "+f"(m4[0]), "+f"(m4[1]), "+f"(m4[2]), "+f"(m4[3])::"memory");
+      tmem_ld_wait(sr[2]);
+      tmem_ld_wait(sr[3]);
+      take(2);
+#pragma unroll
+      for (int col = 64; col < 128; col += 8)
 #pragma unroll
         for (int j = 0; j < 4; ++j) m4[j] = fmax3(m4[j], x[col + j], x[col + 4 + j]);
       const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
@@ -425,31 +443,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (rare) passes that need it, both halves of P are released after it.
       const bool resc = __any_sync(0xffffffffu, rescale_o) && p > 0;
       // p = 2^(s * scale * log2 e - m): one packed FMA per pair, the row sum in
-      // two packed accumulators; otherwise each 64-key half of P is released to
-      // the MMA warp as soon as it is in TMEM.
+      // two packed accumulators.
       const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-msub, -msub);
       uint64_t acc[2] = {0ull, 0ull};
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      // One pair of P: 2^(s * scale * log2 e - m) for columns 64 half + 2k, +1.
+      auto pair_exp = [&](int half, int k) -> uint32_t {
+        const uint64_t ev = f2_fma(f2_pack(x[half * 64 + 2 * k], x[half * 64 + 2 * k + 1]), sc2, nm2);
+        float p0, p1;
+        if (kPolyEvery > 0 && (k % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+          f2_unpack(ex2_poly2(ev), p0, p1);  // on the FMA pipe
+        } else {
+          float e0, e1;
+          f2_unpack(ev, e0, e1);
+          p0 = ex2_approx(e0);  // on the MUFU
+          p1 = ex2_approx(e1);
+        }
+        acc[k & 1] = f2_add(acc[k & 1], f2_pack(p0, p1));
+        return pack_bf16x2(p0, p1);
+      };
+      // P half 0 is stored, then half 1's first eight pairs are taken while
+      // that store lands (6-8 measured best); half 0 is released after them,
+      // half 1 at the end.  In a pass that rescales O both are released after
+      // the rescale.
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const uint64_t ev = f2_fma(f2_pack(x[half * 64 + 2 * k], x[half * 64 + 2 * k + 1]), sc2, nm2);
-          float p0, p1;
-          if (kPolyEvery > 0 && (k % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-            f2_unpack(ex2_poly2(ev), p0, p1);  // on the FMA pipe
-          } else {
-            float e0, e1;
-            f2_unpack(ev, e0, e1);
-            p0 = ex2_approx(e0);  // on the MUFU
-            p1 = ex2_approx(e1);
-          }
-          acc[k & 1] = f2_add(acc[k & 1], f2_pack(p0, p1));
-          pk[k] = pack_bf16x2(p0, p1);
+        for (int k = 0; k < 32; ++k) pk[k] = pair_exp(0, k);
+        tmem_st32(s_addr, pk);
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pk[k] = pair_exp(1, k);
+        if (!resc) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(kPFull + 2 * h));
         }
-        tmem_st32(s_addr + half * 32, pk);
-        if (half == 0 && resc) continue;
-        if (half == 1 && resc) {
+#pragma unroll
+        for (int k = 8; k < 32; ++k) pk[k] = pair_exp(1, k);
+        tmem_st32(s_addr + 32, pk);
+        if (resc) {
           // O_h(p-1) is final here: its product was issued before S_h(p).
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -463,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        if (half == 1 && resc) mbar_arrive(bar(kPFull + 2 * h));
-        mbar_arrive(bar(kPFull + 2 * h + half));
+        if (resc) mbar_arrive(bar(kPFull + 2 * h));
+        mbar_arrive(bar(kPFull + 2 * h + 1));
       }
       {
         float a0, a1;
