@@ -28,6 +28,10 @@
  *     half-split RoPE pairs (t, t + D/2), theta_t = rope_base^(-2t/D).
  *   - D (head_dim) is 64 or 128; Hq % Hkv == 0; 1 <= L; w0 >= 0;
  *     w_pretrained >= 1.  softmax_scale == 0 means 1/sqrt(D).
+ *   - Size limits (JL_ERR_UNSUPPORTED beyond them): L <= 2^30; B and Hkv
+ *     <= 65535; one prefill call's query rows <= 65535 * 128 = 8,388,480
+ *     (longer prompts go in chunks, jl_bifocal_prefill_chunk), with
+ *     Hq * ceil(rows / 128) * B < 2^31.
  *   - Device pointers must be 16-byte aligned.  The caller owns every buffer
  *     (inputs, outputs and scratch); the library never allocates device
  *     memory and never writes its inputs.

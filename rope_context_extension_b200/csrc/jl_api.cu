@@ -67,6 +67,8 @@ void fill_theta(double* theta, int D, double base) {
   for (int t = 0; t < D / 2; ++t) theta[t] = std::pow(base, -2.0 * t / D);
 }
 
+constexpr int kMaxGridYZ = 65535;  // CUDA's limit on a grid's y and z dimensions
+
 int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained, double rope_base, int mode) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || w0 < 0 || w_pretrained < 1) return JL_ERR_INVALID_ARG;
   if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return JL_ERR_INVALID_ARG;
@@ -74,6 +76,7 @@ int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained
   if (Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
   if (L > (1 << 30)) return JL_ERR_UNSUPPORTED;
+  if (B > kMaxGridYZ || Hkv > kMaxGridYZ) return JL_ERR_UNSUPPORTED;  // grid y / z dimensions
   return JL_OK;
 }
 
@@ -227,6 +230,10 @@ int problem_checks(const PrefillProblem& pp, int w0, int w_pretrained, double ro
   int st = common_checks(pp.B, pp.Lk(), pp.Hq, pp.Hkv, pp.D, w0, w_pretrained, rope_base, mode);
   if (st != JL_OK) return st;
   if (pp.q_off < 0 || pp.Lq < 1 || pp.k_rows < pp.Lk()) return JL_ERR_INVALID_ARG;
+  // attention grid: (query-head groups, 128-row query blocks, batch), with a
+  // 32-bit linear CTA index
+  const int64_t blocks = ((int64_t)pp.Lq + 127) / 128;
+  if (blocks > kMaxGridYZ || (int64_t)pp.Hq * blocks * pp.B > INT32_MAX) return JL_ERR_UNSUPPORTED;
   if (!pp.q || !pp.k || !pp.v) return JL_ERR_INVALID_ARG;
   if (!aligned16(pp.q) || !aligned16(pp.k) || !aligned16(pp.v)) return JL_ERR_ALIGNMENT;
   return JL_OK;

@@ -137,6 +137,11 @@ def _decode(lib, q=A, k=A, v=A, cache_len=256, o=A, lse=None, B=1, L=256, Hq=4, 
 
 def test_prefill_argument_errors(lib):
     assert _prefill(lib, D=96) == JL_ERR_UNSUPPORTED
+    # grid limits: 65535 query blocks of 128 rows, B <= 65535, a 32-bit CTA index
+    assert _prefill(lib, L=65535 * 128 + 1, w0=0) == JL_ERR_UNSUPPORTED
+    assert _prefill(lib, B=65536) == JL_ERR_UNSUPPORTED
+    assert _prefill(lib, B=65535, L=65535 * 128, Hq=4, Hkv=2) == JL_ERR_UNSUPPORTED
+    assert _decode(lib, B=65536) == JL_ERR_UNSUPPORTED
     assert _prefill(lib, Hq=3, Hkv=2) == JL_ERR_INVALID_ARG
     assert _prefill(lib, L=0) == JL_ERR_INVALID_ARG
     assert _prefill(lib, w0=-1) == JL_ERR_INVALID_ARG
