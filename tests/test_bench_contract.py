@@ -1,0 +1,60 @@
+"""The bench's one-line JSON contract.
+
+Both arms print exactly one JSON line on stdout with the keys a caller reads:
+the metric and its unit, the whole-job value, the step counts, scaling, dtype,
+data and config; the reference arm (the fp64 oracle on the host cores) adds its
+impl tag, a CPU-baseline description and an e2e block with no host transfers;
+our arm adds the roofline of the dominant kernel, the clocks seen during the
+timed region, the kernel launch count and the end-to-end figure through the
+C ABI with host buffers.
+"""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+BASE_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+             "vs_baseline", "dtype", "data", "config"}
+
+
+def _run(args, timeout):
+    r = subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True, text=True,
+                       timeout=timeout)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, r.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_reference_arm_json_line():
+    d = _run(["--impl", "reference", "--steps", "1", "--warmup", "0"], timeout=600)
+    assert BASE_KEYS <= set(d)
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1
+    assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.gpu
+def test_our_arm_json_line_small():
+    d = _run(["--steps", "3", "--warmup", "3", "--prefill-len", "8192", "--decode-len", "8192", "--cpu-seconds", "2",
+              "--no-split", "--no-ie"], timeout=900)
+    assert BASE_KEYS <= set(d)
+    assert d["n_gpus"] == 1 and d["steps"] == 3 and d["warmup"] == 3 and d["scaling"] == "weak"
+    assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["dtype"] == "bf16"
+    roof = d["roofline"]
+    assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s" and roof["peak"] > 0
+    assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-3
+    e2e = d["e2e"]
+    assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] > 0 and e2e["d2h_bytes_per_step"] > 0
+    assert d["gpu_launches"] > 0
+    assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
+    dec = d["decode"]
+    assert dec["roofline"]["bound"] == "hbm" and dec["value"] > 0
