@@ -136,6 +136,36 @@ def test_decode_cases(B, Lmax, L, Hq, Hkv, D, W, w0, mode, outl):
     assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"decode L{L}")
 
 
+def test_decode_one_million_keys_group_32():
+    # Long context: a cache of 2^20 keys with w_pretrained 32768 gives G = 32,
+    # so positions pass 2^20 and remote distances span the whole pretrained
+    # window.  Two KV heads keep the cache at 1 GiB.
+    L, W, w0 = 1 << 20, 32768, 4096
+    q, kc, vc = synthetic.decode_inputs(1, L, 8, 2, 128, seed=3, outlier_frac=0.01)
+    o, lse, err = run_decode(q, kc, vc, L=L, w0=w0, W=W, base=1e6)
+    assert err == 0
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+    assert jo.group_size(L, W) == 32
+    o_ref, lse_ref = jo.decode(q.float().numpy(), kc.float().numpy(), vc.float().numpy(), p)
+    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, "decode 1M keys, G 32")
+
+
+def test_prefill_group_32_sampled_rows():
+    # G = 32 (L 32768, w_pretrained 1024): every remote key block maps 32 keys to
+    # one position; sampled rows include the band and tile edges.
+    L, W, w0 = 32768, 1024, 700
+    q, k, v = synthetic.prefill_inputs(1, L, 4, 1, 128, seed=9)
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6)
+    assert err == 0
+    rows = sample_rows(L, w0, 96, seed=2)
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+    assert jo.group_size(L, W) == 32
+    ref = oracle_prefill_rows(q, k, v, rows, [0, 3], p)
+    for h in (0, 3):
+        o_ref, lse_ref = ref[h]
+        assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref, f"G 32 h{h}")
+
+
 @pytest.mark.parametrize("B", [1, 8])
 def test_decode_full_size(B):
     # Qwen3-4B shape: 32 q heads / 8 kv heads, d 128, cache of 131072 keys, G 4, w0 4096
