@@ -11,6 +11,7 @@ import pytest
 import torch
 
 from oracle import jetlong_oracle as jo
+from rope_context_extension_b200 import jetlong as jl
 from rope_context_extension_b200 import synthetic
 from tests.gpu_helpers import (LSE_MAX_ABS, LSE_MAX_ABS_FP16_OUTLIERS, assert_close, oracle_prefill_rows,
                                run_decode, run_prefill, sample_rows)
@@ -250,3 +251,31 @@ def test_prefill_split_mode_full_size_sampled():
     for h in heads:
         o_ref, lse_ref = ref[h]
         assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref, f"split 128k h{h}")
+
+
+@pytest.mark.parametrize("split", [False, True])
+def test_two_stage_prefill_equals_fused_call(split):
+    # jl_prefill_correction then jl_prefill_attention (the two stages the fused
+    # entry point launches) give the same bits, and one correction pass serves
+    # repeated attention calls (the workspace is only read by the attention).
+    B, L, Hq, Hkv, D, W, w0 = 2, 900, 8, 2, 128, 250, 180
+    dev = torch.device("cuda")
+    q, k, v = (t.to(dev) for t in synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=17, outlier_frac=0.01))
+    mode = jl.JL_QSHIFT_SELF_EXTEND | (jl.JL_REMOTE_SPLIT if split else 0)
+    ws = torch.empty(jl.jl_prefill_workspace_bytes(B, L, Hq, Hkv, D) * (2 if split else 1), dtype=torch.uint8,
+                     device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    o1, l1 = torch.empty_like(q), torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    jl.jl_bifocal_prefill(q, k, v, o1, l1, w0=w0, w_pretrained=W, rope_base=1e4, mode=mode, workspace=ws,
+                          dev_error=err)
+    ws.fill_(0x5A)  # the stages must not depend on what the fused call left behind
+    jl.jl_prefill_correction(q, k, w0=w0, w_pretrained=W, rope_base=1e4, mode=mode, workspace=ws)
+    outs = []
+    for _ in range(2):
+        o2, l2 = torch.empty_like(q), torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+        jl.jl_prefill_attention(q, k, v, o2, l2, w0=w0, w_pretrained=W, mode=mode, workspace=ws, dev_error=err)
+        outs.append((o2, l2))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for o2, l2 in outs:
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
