@@ -40,7 +40,10 @@
  *     Device-side failures (a pipeline wait that ran out of time) are written
  *     to *dev_error (a device int, may be NULL) as a non-zero value; the
  *     outputs are then invalid.
- *   - Reentrant; no global state beyond cached kernel attributes.
+ *   - Reentrant; no global state beyond cached kernel attributes, with one
+ *     exception: jl_bifocal_decode_noalloc keeps its scratch in a fixed device
+ *     array inside the library, shared by every call on a device, so its
+ *     calls must be ordered on the GPU (see that entry).
  */
 #ifndef JL_API_H
 #define JL_API_H
@@ -299,15 +302,6 @@ int jl_decode_combine(const void* o_parts, const float* lse_parts, int parts, vo
                       int head_dim, void* stream);
 
 /*
- * Diagnostic: evaluates, on the device, the FMA-pipe exponential that the
- * prefill softmax can use for part of each row (Cody-Waite reduction plus a
- * fitted degree-3 polynomial; off by default) and CUDA's exp2f on the same n
- * inputs (device arrays), so its error can be checked.  Not part of the
- * attention path.
- */
-int jl_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, void* stream);
-
-/*
  * Self-test of the failure path every pipeline wait shares (no counterpart on
  * the pages): one tiny kernel waits, with the same bounded mbarrier wait, on a
  * barrier that nothing completes.  After timeout_s seconds (0 < timeout_s <= 10)
@@ -328,16 +322,21 @@ int jl_wait_timeout_check(int* dev_error, double timeout_s, void* stream);
  * this is an interface convenience of this library.
  *   Same arguments, layouts, results and errors as jl_bifocal_decode, minus
  *   the workspace.  Scratch lives in a fixed 4 MiB device array inside the
- *   library (held on every GPU that loads the library until exit); a problem
- *   whose decode scratch (jl_decode_workspace_bytes) exceeds 4 MiB is rejected
+ *   library (held on every GPU that loads the library until exit), laid out
+ *   for the split count the call uses; when that layout would not fit, the
+ *   call runs with fewer splits (same results up to the order of the final
+ *   sum).  A problem that does not fit with one split per (sequence, KV head)
+ *   -- B * Hq * (4 * D + 8) + 4 * B * Hkv bytes plus alignment above 4 MiB,
+ *   e.g. more than 126 sequences of 64 query heads at D = 128 -- is rejected
  *   with JL_ERR_WORKSPACE before any launch.
  *   All calls on a device share that array and it keeps the last call's
  *   contents: calls that overlap on the GPU race and give wrong results, so
  *   order them on one stream (or with events).  The ticket counters are
  *   cleared with cudaMemsetAsync before every launch.
- *   The first call on a device looks up the array's address (cudaGetSymbolAddress,
- *   with that device current) and caches it; make that first call before any
- *   stream capture.  Nothing allocates device memory.
+ *   The first call on a device (and the first after cudaDeviceReset) looks up
+ *   the array's address (cudaGetSymbolAddress, with that device current) and
+ *   caches it; make that first call before any stream capture.  Nothing
+ *   allocates device memory.
  * Launches one memset and one kernel.
  */
 int jl_bifocal_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,

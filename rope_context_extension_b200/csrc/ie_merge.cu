@@ -79,22 +79,6 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const __grid_constant_
   if (lane == 0 && a.lse != nullptr) a.lse[row] = M + logf(den);
 }
 
-// Evaluates the FMA-pipe exponential used by the prefill softmax next to CUDA's
-// exp2f on the same inputs (a check of the polynomial, not a hot path).
-__global__ void exp2_poly_check_kernel(const float* x, float* y_poly, float* y_ref, int n) {
-  const int i2 = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i2 >= n) return;
-  const float a = x[i2], b = (i2 + 1 < n) ? x[i2 + 1] : 0.f;
-  float p0, p1;
-  f2_unpack(ex2_poly2(f2_pack(a, b)), p0, p1);
-  y_poly[i2] = p0;
-  y_ref[i2] = exp2f(a);
-  if (i2 + 1 < n) {
-    y_poly[i2 + 1] = p1;
-    y_ref[i2 + 1] = exp2f(b);
-  }
-}
-
 // Exercises the pipelines' bounded wait on a barrier that nothing completes:
 // warp 0 waits until its limit runs out (it must return false and write the
 // timeout code), warp 1 waits on a second such barrier and must give up as soon
@@ -119,12 +103,6 @@ __global__ void wait_timeout_check_kernel(int* dev_error, unsigned long long tim
 
 cudaError_t launch_wait_timeout_check(int* dev_error, unsigned long long timeout_ns, cudaStream_t stream) {
   wait_timeout_check_kernel<<<1, 64, 0, stream>>>(dev_error, timeout_ns);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream) {
-  const int pairs = (n + 1) / 2;
-  exp2_poly_check_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y_poly, y_ref, n);
   return cudaGetLastError();
 }
 

@@ -479,10 +479,16 @@ size_t jl_decode_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {
 namespace {
 
 // Shared by the uniform-length and the varlen decode entry points.
+// compact = false: the workspace has the layout jl_decode_workspace_bytes sizes
+// (room for decode_splits_max splits).  compact = true (fixed scratch of the
+// no-allocation entry point): the layout holds exactly the split count this
+// call uses, which is lowered until that layout fits in workspace_bytes, and
+// the ticket counters are cleared on the stream before the launch.
 int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len,
                   const int32_t* seq_lens, int L, void* o, float* lse, int B, int Hq, int Hkv, int D, int w0,
                   int w_pretrained, double rope_base, float softmax_scale, int mode, void* workspace,
-                  size_t workspace_bytes, int* dev_error, void* stream, int key_off = 0, int L_total = 0) {
+                  size_t workspace_bytes, int* dev_error, void* stream, int key_off = 0, int L_total = 0,
+                  bool compact = false) {
   int st = common_checks(B, L_total > 0 ? L_total : L, Hq, Hkv, D, w0, w_pretrained, rope_base, mode);
   if (st == JL_OK && L < 1) st = JL_ERR_INVALID_ARG;
   if (st != JL_OK) return st;
@@ -494,8 +500,11 @@ int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64
     return JL_ERR_ALIGNMENT;
   const int tk_keys = jl::decode_tile_keys();
   const int ntiles = (L + tk_keys - 1) / tk_keys;
-  const int splits = decode_splits(B, Hkv, ntiles);
-  const DecodeLayout lay = decode_layout(B, Hq, Hkv, D, decode_splits_max(B, Hkv));
+  int splits = decode_splits(B, Hkv, ntiles);
+  if (compact) {
+    while (splits > 1 && decode_layout(B, Hq, Hkv, D, splits).total > workspace_bytes) --splits;
+  }
+  const DecodeLayout lay = decode_layout(B, Hq, Hkv, D, compact ? splits : decode_splits_max(B, Hkv));
   if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
 
@@ -529,11 +538,31 @@ int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64
   a.qshift = mode & JL_QSHIFT_SELF_EXTEND;
   a.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
   fill_theta(a.theta, D, rope_base);
-  if (jl::launch_decode(tk, tv, a, D, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (compact && cudaMemsetAsync(a.counters, 0, (size_t)B * Hkv * sizeof(int), s) != cudaSuccess)
+    return JL_ERR_CUDA;
+  if (jl::launch_decode(tk, tv, a, D, s) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
 
 }  // namespace
+
+}  // extern "C"
+
+namespace jl {
+
+int decode_in_fixed_scratch(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                            float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
+                            double rope_base, float softmax_scale, int mode, void* scratch, size_t scratch_bytes,
+                            int* dev_error, void* stream) {
+  return decode_launch(q, k_cache, v_cache, cache_len, nullptr, L, o, lse, B, Hq, Hkv, head_dim, w0, w_pretrained,
+                       rope_base, softmax_scale, mode, scratch, scratch_bytes, dev_error, stream, 0, 0,
+                       /*compact=*/true);
+}
+
+}  // namespace jl
+
+extern "C" {
 
 int jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
                       float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
@@ -578,13 +607,6 @@ int jl_decode_combine(const void* o_parts, const float* lse_parts, int parts, vo
   a.B = B;
   a.Hq = Hq;
   if (jl::launch_lse_combine(a, head_dim, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
-  return JL_OK;
-}
-
-int jl_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, void* stream) {
-  if (!x || !y_poly || !y_ref || n < 1) return JL_ERR_INVALID_ARG;
-  if (jl::launch_exp2_poly_check(x, y_poly, y_ref, n, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return JL_ERR_CUDA;
   return JL_OK;
 }
 

@@ -281,37 +281,4 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// 2^x for two values at once on the FMA / ALU pipes (x <= 128): Cody-Waite range
-// reduction 2^x = 2^n * 2^f, n = floor(x), f in [0, 1) (Cody and Waite, Software
-// Manual for the Elementary Functions), and p(f) = 1 + f (c1 + f (c2 + f c3)), a
-// degree-3 minimax fit of 2^f with p(0) = 1 pinned (csrc/exp2_poly_fit.py; max
-// relative error 8.6e-5).  x <= -127 gives exactly 0.  Used for part of the
-// softmax exponentials so that fewer of them queue on the MUFU.
-__device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-// Nothing here runs on the MUFU / conversion pipe: floor(x) comes from one
-// round-down add of 1.5 * 2^23 (whose low mantissa bits then hold floor(x) in
-// two's complement), the fraction from one exact subtraction, and 2^floor(x)
-// is put in by adding floor(x) << 23 to the bits of p(f).
-__device__ __forceinline__ uint64_t ex2_poly2(uint64_t xv) {
-  float x0, x1;
-  f2_unpack(xv, x0, x1);
-  const uint64_t x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f);  // 1.5 * 2^23
-  const uint64_t j = f2_add_rm(x, magic);                   // 1.5 * 2^23 + floor(x), exactly
-  const uint64_t f = f2_sub(x, f2_sub(j, magic));           // x - floor(x), exact
-  uint64_t p = f2_fma(f, f2_pack(0.0770670399f, 0.0770670399f), f2_pack(0.227644995f, 0.227644995f));
-  p = f2_fma(f, p, f2_pack(0.695116758f, 0.695116758f));
-  p = f2_fma(f, p, f2_pack(1.f, 1.f));
-  float p0, p1, j0, j1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(j, j0, j1);
-  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(j0) << 23));
-  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(j1) << 23));
-  return f2_pack(p0, p1);
-}
-
 }  // namespace jl

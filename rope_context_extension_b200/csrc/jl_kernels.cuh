@@ -72,6 +72,17 @@ int decode_ctas_per_sm();
 // Keys per decode tile (one TMA stage; splits cover whole tiles).
 int decode_tile_keys();
 
+// jl_bifocal_decode with its scratch in a caller-given fixed region of
+// scratch_bytes (the no-allocation entry point): the region is laid out for the
+// split count the call uses, lowered until it fits (JL_ERR_WORKSPACE when even
+// one split per (sequence, KV head) does not), and the ticket counters are
+// cleared on the stream before the launch.  Same argument checks as the public
+// entry points; nothing is launched on an argument error.
+int decode_in_fixed_scratch(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
+                            float* lse, int B, int L, int Hq, int Hkv, int head_dim, int w0, int w_pretrained,
+                            double rope_base, float softmax_scale, int mode, void* scratch, size_t scratch_bytes,
+                            int* dev_error, void* stream);
+
 // Inclusion-exclusion merge of three partial prefill outputs.
 struct MergeArgs {
   const __nv_bfloat16* o_x[3];  // O_A, O_B, O_C [B, L, Hq, D]
@@ -91,7 +102,6 @@ struct CombineArgs {
   int R, B, Hq;
 };
 cudaError_t launch_lse_combine(const CombineArgs& a, int D, cudaStream_t stream);
-cudaError_t launch_exp2_poly_check(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream);
 cudaError_t launch_wait_timeout_check(int* dev_error, unsigned long long timeout_ns, cudaStream_t stream);
 
 // Base RoPE of one new token per sequence and its append to the KV cache.

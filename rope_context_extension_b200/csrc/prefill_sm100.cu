@@ -42,12 +42,6 @@ constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
 constexpr int kLowRegs = 104;     // warpgroup 0: TMA producer, MMA issuer
 constexpr int kHighRegs = 200;    // warpgroups 1-2: softmax
-// kPolyEvery > 0 sends one pair of exponentials in every kPolyEvery to the FMA
-// pipe (ex2_poly2, which uses no MUFU or conversion instruction) instead of the
-// MUFU.  Measured at the 128K workload: one pair in four 1026-1030 TFLOP/s and
-// one in eight 1006-1016, against 1031 with every exponential on the MUFU.  The
-// softmax is bound by latency, not by MUFU throughput, so it is off.
-constexpr int kPolyEvery = 0;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kChunkBytes = 128 * 128;  // one 128-row x 128-byte swizzled slab
 
@@ -449,15 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // One pair of P: 2^(s * scale * log2 e - m) for columns 64 half + 2k, +1.
       auto pair_exp = [&](int half, int k) -> uint32_t {
         const uint64_t ev = f2_fma(f2_pack(x[half * 64 + 2 * k], x[half * 64 + 2 * k + 1]), sc2, nm2);
-        float p0, p1;
-        if (kPolyEvery > 0 && (k % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-          f2_unpack(ex2_poly2(ev), p0, p1);  // on the FMA pipe
-        } else {
-          float e0, e1;
-          f2_unpack(ev, e0, e1);
-          p0 = ex2_approx(e0);  // on the MUFU
-          p1 = ex2_approx(e1);
-        }
+        float e0, e1;
+        f2_unpack(ev, e0, e1);
+        const float p0 = ex2_approx(e0), p1 = ex2_approx(e1);  // on the MUFU
         acc[k & 1] = f2_add(acc[k & 1], f2_pack(p0, p1));
         return pack_bf16x2(p0, p1);
       };

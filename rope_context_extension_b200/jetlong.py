@@ -19,7 +19,7 @@ __all__ = [
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
     "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes", "jl_bifocal_prefill_ie", "jl_bifocal_decode_range",
-    "jl_decode_combine", "jl_exp2_poly_check", "jl_wait_timeout_check", "jl_prefill_tile_classes",
+    "jl_decode_combine", "jl_wait_timeout_check", "jl_prefill_tile_classes",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
     "jl_prefill_attention", "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append",
     "jl_prefill_chunk_workspace_bytes", "jl_bifocal_prefill_chunk", "jl_prefill_ie_workspace_bytes",
-    "jl_bifocal_prefill_ie", "jl_bifocal_decode_range", "jl_decode_combine", "jl_exp2_poly_check",
+    "jl_bifocal_prefill_ie", "jl_bifocal_decode_range", "jl_decode_combine",
     "jl_wait_timeout_check", "jl_prefill_tile_classes",
 )
 
@@ -101,8 +101,6 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_decode_range.restype = c_i
     L.jl_decode_combine.argtypes = [c_p, c_p, c_i, c_p, c_p, c_i, c_i, c_i, c_p]
     L.jl_decode_combine.restype = c_i
-    L.jl_exp2_poly_check.argtypes = [c_p, c_p, c_p, c_i, c_p]
-    L.jl_exp2_poly_check.restype = c_i
     L.jl_wait_timeout_check.argtypes = [c_p, c_d, c_p]
     L.jl_wait_timeout_check.restype = c_i
     _lib = L
@@ -396,16 +394,6 @@ def jl_decode_combine(o_parts, lse_parts, o, lse, stream=None):
         _check_tensor(lse, "lse", torch.float32, (B, Hq))
     st = lib().jl_decode_combine(_ptr(o_parts), _ptr(lse_parts), R, _ptr(o), _ptr(lse), B, Hq, D, _stream(stream))
     _check(st, "jl_decode_combine")
-
-
-def jl_exp2_poly_check(x):
-    """(polynomial 2^x, CUDA exp2f) on the device for a float32 CUDA tensor x."""
-    import torch
-    _check_tensor(x, "x", torch.float32)
-    yp = torch.empty_like(x)
-    yr = torch.empty_like(x)
-    _check(lib().jl_exp2_poly_check(_ptr(x), _ptr(yp), _ptr(yr), x.numel(), _stream(None)), "jl_exp2_poly_check")
-    return yp, yr
 
 
 def jl_wait_timeout_check(dev_error, timeout_s: float = 0.2, stream=None):
