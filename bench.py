@@ -3,14 +3,18 @@
 One step = one pass of the whole hot path over one batch of synthetic input:
   * prefill of the Qwen3-8B-shaped layer at 128K (batch 1, 32 q heads / 8 kv
     heads, head_dim 128, RoPE base 1e6, L 131072, w_pretrained 32768 -> G 4,
-    w0 4096): correction pass + fused tcgen05 attention;
+    w0 4096) through the default path: one fused tcgen05 kernel that applies
+    the correction rotations itself and carries remote scores as fp16 hi + lo
+    products (the path held to the oracle's tolerances on every workload);
   * decode of the Qwen3-4B-shaped layer at 128K (32 / 8 heads, head_dim 128,
     batch 8, cache of 131072 base-rotated keys, G 4, w0 4096).
 `value` is the prefill TFLOP/s (algorithmic 4 * B * Hq * d * L(L+1)/2 per
 step, summed over ranks, divided by the max-over-ranks device time of the
 prefill calls); the decode GB/s (K and V bytes read once) is reported beside
-it.  Inputs are larger than L2 (1 GiB Q, 4 GiB KV cache), so no flush runs
-between steps.
+it, and so are the other prefill paths (single fp16 product, pre-rotated key
+rows, the three-call inclusion-exclusion formulation, plain RoPE), the
+Qwen3-1.7B 64K and tiny workloads and the length / band sweep.  Inputs are
+larger than L2 (1 GiB Q, 4 GiB KV cache), so no flush runs between steps.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
 
@@ -40,6 +44,11 @@ PREFILL = dict(workload="qwen3-8b-shaped bifocal prefill, single layer", B=1, L=
                W=32768, w0=4096, base=1e6)
 DECODE = dict(workload="qwen3-4b-shaped bifocal decode", B=8, L=131072, Hq=32, Hkv=8, D=128, W=32768, w0=4096,
               base=1e6)
+# the other workloads of the method's evaluation shapes, reported beside the headline
+PREFILL_1P7B = dict(workload="qwen3-1.7b-shaped bifocal prefill, single layer", B=1, L=65536, Hq=16, Hkv=8, D=128,
+                    W=32768, w0=4096, base=1e6)
+PREFILL_TINY = dict(workload="tiny bifocal prefill", B=1, L=512, Hq=2, Hkv=1, D=64, W=128, w0=32, base=1e4)
+SWEEP_L = (16384, 32768, 32769, 49152, 100003, 131072)  # qwen3-4b shape, w0 in {0, 4096, L}, 1% x8 key outliers
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -64,7 +73,7 @@ def load_peaks():
 # Source files that determine each timed kernel's code and launch shape; a
 # traffic figure is used only while these hash to the value stored with it.
 KERNEL_SOURCES = {
-    "prefill_attention": ["prefill_sm100.cu", "jl_common.cuh", "jl_kernels.cuh", "jl_api.cu"],
+    "prefill_attention": ["prefill_hilo_sm100.cu", "jl_common.cuh", "jl_kernels.cuh", "jl_api.cu"],
     "decode": ["decode_sm100.cu", "jl_common.cuh", "jl_kernels.cuh", "jl_api.cu"],
 }
 
@@ -196,6 +205,33 @@ def gen_on_device(shape, seed, dev):
     return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
 
 
+def scale_outliers_on_device(k, frac, seed, scale=8.0):
+    """Multiply a seeded `frac` share of the (b, j, kv-head) rows of k by `scale`."""
+    import torch
+    B, L, H, _ = k.shape
+    g = torch.Generator(device=k.device).manual_seed(seed)
+    n = max(1, int(round(frac * B * L * H)))
+    idx = torch.randperm(B * L * H, generator=g, device=k.device)[:n]
+    kf = k.view(B * L * H, -1)
+    kf[idx] = (kf[idx].float() * scale).to(torch.bfloat16)
+    return k
+
+
+def executed_prefill_flop(c, jl):
+    """Flop the tensor core executes for one prefill of workload c on the
+    default path: one 128 x 128 tile product (S or P V) is 2 * 128 * 128 * D
+    flop; a local pass issues S once, a remote pass three times (hi + lo),
+    and every pass issues one P V.  Diagnostic beside the algorithmic count."""
+    loc_only, both, rem_only, _ = jl.jl_prefill_tile_classes(c["L"], c["w0"], c["W"])
+    per_tile = 2.0 * 128 * 128 * c["D"]
+    G = jl.jl_group_size(c["L"], c["W"])
+    if G == 1 or c["w0"] >= c["L"]:
+        units = 2.0 * (loc_only + both + rem_only)
+    else:
+        units = 2.0 * (loc_only + both) + 4.0 * (rem_only + both)
+    return per_tile * units * c["B"] * c["Hq"]
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -223,6 +259,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     P, Dc = PREFILL, DECODE
     seed = 1000 * rank
+    SE = jl.JL_QSHIFT_SELF_EXTEND
 
     # prefill buffers (resident in HBM)
     q = gen_on_device((P["B"], P["L"], P["Hq"], P["D"]), seed + 0, dev)
@@ -230,8 +267,6 @@ def run_ours(args):
     v = gen_on_device((P["B"], P["L"], P["Hkv"], P["D"]), seed + 2, dev)
     o = torch.empty_like(q)
     lse = torch.empty(P["B"], P["Hq"], P["L"], dtype=torch.float32, device=dev)
-    ws = torch.empty(jl.jl_prefill_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]), dtype=torch.uint8,
-                     device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     # decode buffers
     dq = gen_on_device((Dc["B"], Dc["Hq"], Dc["D"]), seed + 3, dev)
@@ -242,19 +277,17 @@ def run_ours(args):
     dws = torch.zeros(jl.jl_decode_workspace_bytes(Dc["B"], Dc["L"], Dc["Hq"], Dc["Hkv"], Dc["D"]),
                       dtype=torch.uint8, device=dev)
 
-    pkw = dict(w0=P["w0"], w_pretrained=P["W"], stream=stream)
-
-    def prefill_step(evs=None, w0=None, mode=jl.JL_QSHIFT_SELF_EXTEND, wsp=None):
+    def prefill_step(evs=None, w0=None, mode=SE, wsp=None):
+        # stage 1 (the correction pass) launches nothing in the default mode
         w = P["w0"] if w0 is None else w0
-        wsb = ws if wsp is None else wsp
         if evs:
             evs[0].record(stream)
-        jl.jl_prefill_correction(q, k, w0=w, w_pretrained=P["W"], rope_base=P["base"], mode=mode, workspace=wsb,
+        jl.jl_prefill_correction(q, k, w0=w, w_pretrained=P["W"], rope_base=P["base"], mode=mode, workspace=wsp,
                                  stream=stream)
         if evs:
             evs[1].record(stream)
-        jl.jl_prefill_attention(q, k, v, o, lse, w0=w, w_pretrained=P["W"], mode=mode, workspace=wsb,
-                                dev_error=err, stream=stream)
+        jl.jl_prefill_attention(q, k, v, o, lse, w0=w, w_pretrained=P["W"], rope_base=P["base"], mode=mode,
+                                workspace=wsp, dev_error=err, stream=stream)
         if evs:
             evs[2].record(stream)
 
@@ -291,7 +324,7 @@ def run_ours(args):
     barrier(world)
     clk = clocks.stop()
     if int(err.item()) != 0:
-        raise RuntimeError("device pipeline timeout flag set during the timed region")
+        raise RuntimeError(f"device error {int(err.item())} during the timed region")
 
     total_ms = t0.elapsed_time(t1)
     corr_ms = sum(e[0].elapsed_time(e[1]) for e in pev) / K
@@ -307,10 +340,9 @@ def run_ours(args):
     dbytes = decode_bytes(Dc)
     value = weak_scaling_value(flop, world, pre_ms_max) / 1e12
     attn_tflops = flop / (attn_ms_max * 1e-3) / 1e12
-    dec_gbs = weak_scaling_value(dbytes, world, dec_ms_max) / 1e9
     dec_gbs_kernel = dbytes / (dec_ms_max * 1e-3) / 1e9
+    exec_flop = executed_prefill_flop(P, jl)
 
-    # plain causal RoPE from the same kernels (w0 = L), measured after the timed region
     def time_calls(fn, reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         fn()
@@ -323,8 +355,8 @@ def run_ours(args):
         return a.elapsed_time(b) / reps
 
     # decode on its own, launches back to back as a serving loop issues them
-    # (the in-step decode above runs right after a 138 ms prefill, under its
-    # power cap); B 8 and B 1 against the same 128K cache
+    # (the in-step decode above runs right after the prefill, under its power
+    # cap); B 8 and B 1 against the same 128K cache
     def decode_loop(bsz, seconds=0.6):
         qb, kb, vb, ob, lb = dq[:bsz], kc[:bsz], vc[:bsz], do[:bsz], dlse[:bsz]
 
@@ -362,28 +394,93 @@ def run_ours(args):
         dloop8 = decode_loop(Dc["B"])
         dloop1 = decode_loop(1)
     if int(err.item()) != 0:
-        raise RuntimeError("device pipeline timeout flag set during the decode loops")
+        raise RuntimeError(f"device error {int(err.item())} during the decode loops")
 
+    # plain causal RoPE from the same library entry points (w0 = L)
     plain_pre_ms = time_calls(lambda: prefill_step(w0=P["L"]), max(2, K // 2))
     plain_dec_ms = time_calls(lambda: decode_step(w0=Dc["L"]), max(2, K // 2))
-    # the pages' unfused three-call inclusion-exclusion formulation, same inputs
-    ie_ms = None
+    # the other prefill paths on the same inputs
+    ws_opt = torch.empty(jl.jl_prefill_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]), dtype=torch.uint8,
+                         device=dev)
+    paths = {}
+    for name, flag in (("fp16_single_product", jl.JL_PREFILL_FP16),
+                       ("prerotated_keys", jl.JL_PREFILL_PREROTATED_K)):
+        if args.no_variants:
+            break
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ms = time_calls(lambda: prefill_step(mode=SE | flag, wsp=ws_opt), 2)
+        prefill_step(evs, mode=SE | flag, wsp=ws_opt)
+        torch.cuda.synchronize()
+        paths[name] = {"ms": round(ms, 3), "tflops": round(flop / (ms * 1e-3) / 1e12, 2),
+                       "correction_ms": round(evs[0].elapsed_time(evs[1]), 3),
+                       "attention_ms": round(evs[1].elapsed_time(evs[2]), 3),
+                       "speed_vs_default": round(pre_ms_max / ms, 3)}
+    del ws_opt
+    ie = None
     if not args.no_ie:
         ws3 = torch.empty(jl.jl_prefill_ie_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]),
                           dtype=torch.uint8, device=dev)
         ie_ms = time_calls(lambda: jl.jl_bifocal_prefill_ie(q, k, v, o, lse, w0=P["w0"], w_pretrained=P["W"],
                                                             rope_base=P["base"], workspace=ws3, dev_error=err,
                                                             stream=stream), 2)
+        ie = {"ms": round(ie_ms, 3), "tflops": round(flop / (ie_ms * 1e-3) / 1e12, 2),
+              "fused_speedup": round(ie_ms / pre_ms_max, 3)}
         del ws3
-    # split-precision remote products (for inputs with dominant large-norm keys)
-    split_pre_ms = None
-    if not args.no_split:
-        ws2 = torch.empty(2 * ws.numel(), dtype=torch.uint8, device=dev)
-        split_pre_ms = time_calls(lambda: prefill_step(mode=jl.JL_QSHIFT_SELF_EXTEND | jl.JL_REMOTE_SPLIT, wsp=ws2),
-                                  2)
-        del ws2
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error {int(err.item())} in the prefill variants")
 
-    # end to end through the public API: pinned host inputs in, result out, every step
+    # the other workloads: Qwen3-1.7B 64K and tiny prefill (bifocal and plain),
+    # and the length / band sweep (prefill and B 1 decode, 1% x8 key outliers)
+    others = None
+    if not args.no_other_workloads:
+        others = {}
+        for c in (PREFILL_1P7B, PREFILL_TINY):
+            q2 = gen_on_device((c["B"], c["L"], c["Hq"], c["D"]), seed + 11, dev)
+            k2 = gen_on_device((c["B"], c["L"], c["Hkv"], c["D"]), seed + 12, dev)
+            v2 = gen_on_device((c["B"], c["L"], c["Hkv"], c["D"]), seed + 13, dev)
+            o2 = torch.empty_like(q2)
+            l2 = torch.empty(c["B"], c["Hq"], c["L"], dtype=torch.float32, device=dev)
+            res = {}
+            for tag, w0 in (("bifocal", c["w0"]), ("plain", c["L"])):
+                reps = 3 if c["L"] > 8192 else 200
+                ms = time_calls(lambda: jl.jl_bifocal_prefill(q2, k2, v2, o2, l2, w0=w0, w_pretrained=c["W"],
+                                                              rope_base=c["base"], dev_error=err, stream=stream),
+                                reps)
+                f = prefill_flop(c)
+                res[tag] = {"ms": round(ms, 4), "tflops": round(f / (ms * 1e-3) / 1e12, 2),
+                            "tokens_per_s": round(c["B"] * c["L"] / (ms * 1e-3), 1)}
+            res["shape"] = {k_: c[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")}
+            others[c["workload"]] = res
+            del q2, k2, v2, o2, l2
+        sweep = []
+        sh = dict(B=1, Hq=32, Hkv=8, D=128, W=32768, base=1e6)
+        dws1 = torch.zeros(jl.jl_decode_workspace_bytes(1, max(SWEEP_L), 32, 8, 128), dtype=torch.uint8, device=dev)
+        for L in SWEEP_L:
+            q2 = gen_on_device((1, L, 32, 128), seed + L, dev)
+            k2 = scale_outliers_on_device(gen_on_device((1, L, 8, 128), seed + L + 1, dev), 0.01, seed + 7)
+            v2 = gen_on_device((1, L, 8, 128), seed + L + 2, dev)
+            o2 = torch.empty_like(q2)
+            l2 = torch.empty(1, 32, L, dtype=torch.float32, device=dev)
+            qd1, od1 = q2[:, L - 1].contiguous(), torch.empty(1, 32, 128, dtype=torch.bfloat16, device=dev)
+            ld1 = torch.empty(1, 32, dtype=torch.float32, device=dev)
+            for w0 in (0, 4096, L):
+                c = dict(sh, L=L, w0=w0)
+                pms = time_calls(lambda: jl.jl_bifocal_prefill(q2, k2, v2, o2, l2, w0=w0, w_pretrained=sh["W"],
+                                                               rope_base=sh["base"], dev_error=err, stream=stream), 2)
+                dms = time_calls(lambda: jl.jl_bifocal_decode(qd1, k2, v2, od1, ld1, L=L, w0=w0,
+                                                              w_pretrained=sh["W"], rope_base=sh["base"],
+                                                              workspace=dws1, dev_error=err, stream=stream), 20)
+                sweep.append({"L": L, "w0": w0, "G": jl.jl_group_size(L, sh["W"]),
+                              "prefill_ms": round(pms, 3), "prefill_tflops": round(prefill_flop(c) / (pms * 1e-3) / 1e12, 2),
+                              "prefill_tokens_per_s": round(L / (pms * 1e-3), 1),
+                              "decode_ms": round(dms, 4), "decode_gbs": round(decode_bytes(c) / (dms * 1e-3) / 1e9, 1),
+                              "decode_tokens_per_s": round(1 / (dms * 1e-3), 1)})
+            del q2, k2, v2, o2, l2
+        others["length / band sweep (qwen3-4b shape, 1% x8 key outliers, decode B 1)"] = sweep
+        del dws1
+        if int(err.item()) != 0:
+            raise RuntimeError(f"device error {int(err.item())} in the other workloads")
+
     # end to end through the public API: pinned host inputs in, result out, every
     # step.  Pipelined as a serving loop runs it: step i's host-to-device copies
     # (own stream) and step i-1's result copy-back (another stream) overlap the
@@ -403,7 +500,7 @@ def run_ours(args):
 
         def e2e_call(bq, bk, bv, bo):
             jl.jl_bifocal_prefill(bq, bk, bv, bo, lse, w0=P["w0"], w_pretrained=P["W"], rope_base=P["base"],
-                                  workspace=ws, dev_error=err, stream=stream)
+                                  dev_error=err, stream=stream)
 
         def pipelined(reps):
             ev = lambda: torch.cuda.Event()
@@ -464,15 +561,19 @@ def run_ours(args):
                "serial": {"ms_per_step": round(serial_ms, 3),
                           "value": round(world * flop / (serial_ms * 1e-3) / 1e12, 2)}}
         del bufs
+        if int(err.item()) != 0:
+            raise RuntimeError(f"device error {int(err.item())} in the end-to-end loop")
 
     peaks, peak_kind = load_peaks()
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     # the stored traffic figures are per launch of the default (128K) workloads
     traffic = load_traffic() if not (args.prefill_len or args.decode_len or args.decode_batch) else {}
+    sm_ghz = (clk.get("sm_mhz") or 0) / 1e3
+    peak_ghz = (peaks.get("clocks_under_load", {}).get("sm_mhz_median") or 0) / 1e3
     out = None
     if rank == 0:
         # the oracle's CPU baseline is taken on rank 0 of a one-GPU run only
-        cpu = None if (args.no_cpu_baseline or world > 1) else cpu_baseline_sample(seconds=args.cpu_seconds)
+        cpu = None if (args.no_cpu_baseline or world > 1) else cpu_baseline(seconds=args.cpu_seconds)
         out = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -490,7 +591,9 @@ def run_ours(args):
             "prefill": {"ms": round(pre_ms_max, 3), "correction_ms": round(corr_ms, 3),
                         "attention_ms": round(attn_ms_max, 3), "tokens_per_s": round(world * P["L"] * P["B"] /
                                                                                      (pre_ms_max * 1e-3), 1),
-                        "attention_tflops": round(attn_tflops, 2)},
+                        "attention_tflops": round(attn_tflops, 2),
+                        "path": "default: corrections inside the kernel, remote scores Q_hi K_hi + Q_hi K_lo + "
+                                "Q_lo K_hi (fp16 hi + lo), no workspace"},
             "decode": {"value": dloop8["gbs_all_ranks"], "unit": "GB/s", "ms": dloop8["ms"],
                        "tokens_per_s": dloop8["tokens_per_s"], "B": Dc["B"],
                        "timing": f"{dloop8['reps']} launches back to back between two CUDA events, mean period",
@@ -506,24 +609,29 @@ def run_ours(args):
                        "in_step": {"ms": round(dec_ms_max, 4), "gbs": round(dec_gbs_kernel, 1),
                                    "frac": round(dec_gbs_kernel / peaks["hbm_gbs"], 4),
                                    "note": "timed inside the step, right after the prefill kernel"}},
-            "prefill_inclusion_exclusion_3pass": None if ie_ms is None else {
-                "ms": round(ie_ms, 3), "tflops": round(flop / (ie_ms * 1e-3) / 1e12, 2),
-                "fused_speedup": round(ie_ms / pre_ms_max, 3)},
-            "prefill_split_precision": None if split_pre_ms is None else {
-                "ms": round(split_pre_ms, 3), "tflops": round(flop / (split_pre_ms * 1e-3) / 1e12, 2)},
+            "prefill_other_paths": paths,
+            "prefill_inclusion_exclusion_3pass": ie,
             "plain_rope_same_kernels": {
                 "prefill_ms": round(plain_pre_ms, 3),
                 "prefill_tflops": round(flop / (plain_pre_ms * 1e-3) / 1e12, 2),
                 "decode_ms": round(plain_dec_ms, 4),
                 "decode_gbs": round(dbytes / (plain_dec_ms * 1e-3) / 1e9, 1),
             },
+            "other_workloads": others,
             "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": tensor_peak,
                          "unit": "TFLOP/s", "frac": round(attn_tflops / tensor_peak, 4),
                          "traffic": traffic.get("prefill_attention", {}).get("bytes_per_launch"),
-                         "kernel": "bifocal_prefill_kernel<128>",
-                         "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a multi-second loop)"},
+                         "kernel": "bifocal_prefill_hilo_kernel<128, true, 0>",
+                         "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a multi-second loop)",
+                         "executed_tflops": round(exec_flop / (attn_ms_max * 1e-3) / 1e12, 2),
+                         "executed_frac": round(exec_flop / (attn_ms_max * 1e-3) / 1e12 / tensor_peak, 4),
+                         "executed_note": "tensor-core flop actually issued: three score products per remote tile "
+                                          "(hi + lo), one per local tile, one P V per tile",
+                         "per_ghz": {"kernel_tflops_per_sm_ghz": round(attn_tflops / sm_ghz, 1) if sm_ghz else None,
+                                     "peak_tflops_per_sm_ghz": round(tensor_peak / peak_ghz, 1) if peak_ghz else None,
+                                     "note": "TFLOP/s divided by the median SM clock sampled while each ran"}},
             "e2e": e2e,
-            "gpu_launches": K * 4,
+            "gpu_launches": K * 2,
             "gpu_launches_decode_loops": dloop8["reps"] + dloop1["reps"],
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -532,7 +640,6 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return out
-
 
 # ---------------------------------------------------------------------------
 # oracle timing (CPU baseline and the reference arm)
@@ -582,7 +689,7 @@ def _cores():
 def cpu_baseline_sample(seconds=15.0):
     """The oracle on batches of random query rows (new rows each batch) until
     about `seconds` of CPU time have been spent; TFLOP/s from the algorithmic
-    flop of the rows done."""
+    flop of the rows done (each row i costs 4 d (i + 1) flop per head)."""
     _oracle_rows_timed(2, seed=7)  # warm-up (thread pool, first-touch)
     flop_sum, t_sum, rows, batch, seed = 0.0, 0.0, 0, 8, 1
     while t_sum < seconds:
@@ -592,9 +699,47 @@ def cpu_baseline_sample(seconds=15.0):
         rows += batch
         seed += 1
         batch = int(max(8, min(256, batch * max(1.0, (seconds - t_sum) / max(dt, 1e-3)) * 0.5)))
-    return {"value": round(flop_sum / t_sum / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+    return flop_sum / t_sum / 1e12, rows, t_sum
+
+
+def cpu_baseline(seconds=15.0):
+    """The fp64 oracle, as it stands, on the host cores: a bounded sample of the
+    128K prefill workload (all cores, and again on one core), the full prefill
+    time extrapolated from it by the causal row-cost sum, and the B 1 decode of
+    the 128K decode workload timed in full."""
+    import numpy as np
+    import torch
+    from oracle import jetlong_oracle as jo
+    tf, rows, t_sum = cpu_baseline_sample(seconds)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            tf1, rows1, t1 = cpu_baseline_sample(max(2.0, seconds / 3))
+    except ImportError:  # pragma: no cover - threadpoolctl is in the image
+        tf1, rows1, t1 = None, 0, 0.0
+    full_s = prefill_flop(PREFILL) / (tf * 1e12)
+    # decode, B 1, 128K cache, every head and key
+    Dc = DECODE
+    g = torch.Generator("cpu").manual_seed(3)
+    dq = torch.randn(1, Dc["Hq"], Dc["D"], generator=g).to(torch.bfloat16).double().numpy()
+    kc = torch.randn(1, Dc["L"], Dc["Hkv"], Dc["D"], generator=g).to(torch.bfloat16).double().numpy()
+    vc = torch.randn(1, Dc["L"], Dc["Hkv"], Dc["D"], generator=g).to(torch.bfloat16).double().numpy()
+    p = jo.BifocalParams(L=Dc["L"], w0=Dc["w0"], w_pretrained=Dc["W"], base=Dc["base"])
+    t = time.perf_counter()
+    jo.decode(dq, kc, vc, p)
+    dec_s = time.perf_counter() - t
+    dbytes = decode_bytes(dict(Dc, B=1))
+    return {"value": round(tf, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
             "sample": f"fp64 oracle, {rows} random query rows x 4 q heads of one KV head of the 128K prefill "
-                      f"workload, {t_sum:.1f} s; TFLOP/s from the algorithmic flop of those rows"}
+                      f"workload, {t_sum:.1f} s; TFLOP/s from the algorithmic flop of those rows",
+            "one_core": None if tf1 is None else {"value": round(tf1, 6), "unit": "TFLOP/s", "cores": 1,
+                                                 "sample": f"{rows1} rows, {t1:.1f} s"},
+            "prefill_128k_full_s_extrapolated": round(full_s, 1),
+            "extrapolation": "full prefill time = its algorithmic flop (sum over rows of 4 d (i + 1) per head) / "
+                             "the sampled rate; extrapolated, not run",
+            "decode_128k_b1_full": {"s": round(dec_s, 3), "gbs": round(dbytes / dec_s / 1e9, 4),
+                                    "tokens_per_s": round(1.0 / dec_s, 4),
+                                    "sample": "the whole decode (32 q heads, 131072 keys), timed in full"}}
 
 
 def run_reference(args):
@@ -640,7 +785,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-split", action="store_true", help="skip the split-precision prefill measurement")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the fp16-single-product and pre-rotated-key prefill measurements")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the 1.7B 64K, tiny and length / band sweep measurements")
     ap.add_argument("--no-ie", action="store_true", help="skip the three-call inclusion-exclusion measurement")
     ap.add_argument("--no-decode-loops", action="store_true",
                     help="report the in-step decode time only (profiling runs: no back-to-back decode loops)")

@@ -68,15 +68,33 @@ typedef enum {
 typedef enum { JL_QSHIFT_NONE = 0, JL_QSHIFT_SELF_EXTEND = 1 } jl_qshift;
 
 /*
- * Optional flag OR-ed into `mode` of the prefill and decode entry points.
- * JL_REMOTE_SPLIT: prefill forms remote scores from fp16 hi + lo corrected rows
- * (Q_hi K_hi + Q_hi K_lo + Q_lo K_hi, about 2^-21 relative operand error
- * instead of 2^-12), for inputs where a few keys of large norm dominate the
- * softmax and the fp16 rounding of the default path shows in the LSE.  It runs
- * one query head per CTA and needs twice the prefill workspace.  Decode always
- * carries its corrected operands as hi + lo pairs and ignores the flag.
+ * Optional prefill flags, OR-ed into `mode` (decode ignores them).  The default
+ * prefill (neither flag) applies the correction rotations R(p_q(i) - i) and
+ * R(f(j) - j) inside the attention kernel, in fp32 registers, to the query
+ * block once and to every remote key tile as it streams through shared memory,
+ * and forms remote scores from fp16 hi + lo operands: S = Q_hi K_hi + Q_hi K_lo
+ * + Q_lo K_hi with x = hi + lo to about 22 significant bits, so a score's
+ * rounding error is about 2^-21 |q| |k| (in fp32 accumulation).  It needs no
+ * scratch memory.  Local (base RoPE) scores and P V use the bf16 inputs as
+ * they are.  Corrected values must stay within fp16's range: a query or key
+ * component of magnitude 46340 or more can overflow, which the kernel reports
+ * as device error 3 (results invalid).
+ *
+ * JL_PREFILL_FP16: a correction pass writes R(p_q(i) - i) Q_i and R(f(j) - j) K_j
+ *   to the workspace, rounded once to fp16, and the attention kernel forms each
+ *   remote score with one fp16 product (two query heads per CTA).  Faster, but
+ *   a score's rounding error is about 2^-11 |q| |k|: on rows dominated by one
+ *   key of large norm that shows in the LSE (1e-2 on the pages' outlier
+ *   workload).  Needs jl_prefill_workspace_bytes(...) of scratch.
+ * JL_PREFILL_PREROTATED_K: the default's hi + lo arithmetic, but the key rows'
+ *   hi / lo parts come from a correction pass into the workspace instead of
+ *   being rotated inside the attention kernel (for comparing the two designs;
+ *   same results up to the order of fp32 operations).  Needs scratch.
+ * The two flags are exclusive.  When every pair is local (G = 1 or w0 >= L) no
+ * operand is corrected and every mode runs plain causal RoPE attention on the
+ * bf16 inputs.
  */
-enum { JL_REMOTE_SPLIT = 2 };
+enum { JL_PREFILL_FP16 = 4, JL_PREFILL_PREROTATED_K = 8 };
 
 /* Human-readable name of a status code (static string). */
 const char* jl_status_string(int status);
@@ -114,9 +132,11 @@ int jl_remote_positions(int64_t L, int64_t w0, int64_t w_pretrained, int mode, i
 int jl_prefill_tile_classes(int64_t L, int64_t w0, int64_t w_pretrained, int64_t* counts_out);
 
 /*
- * Scratch bytes jl_bifocal_prefill needs: space for the remote-rotated Q and K
- * rows (2 * B * L * (Hq + Hkv) * D bytes plus alignment); twice this with
- * JL_REMOTE_SPLIT in `mode`.  0 on bad arguments.
+ * Scratch bytes jl_bifocal_prefill may need: the larger of the two opt-in
+ * modes' needs (JL_PREFILL_FP16: fp16 corrected query and key rows, 2 * B * L *
+ * (Hq + Hkv) * D bytes; JL_PREFILL_PREROTATED_K: fp16 hi and lo key rows,
+ * 4 * B * L * Hkv * D bytes; each plus alignment).  The default mode needs
+ * none (pass NULL and 0).  0 on bad arguments.
  */
 size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim);
 
@@ -126,11 +146,16 @@ size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim);
  *   o [B, L, Hq, D] bf16 device (written); lse [B, Hq, L] fp32 device or NULL.
  *   w0: band width of exact base-RoPE scoring (i - j < w0); w0 >= L, or
  *   L <= w_pretrained (G = 1), gives plain causal RoPE attention.
- *   workspace: device scratch of at least jl_prefill_workspace_bytes(...) bytes
- *   (contents on entry do not matter; overwritten).
- * Launches: jl_prefill_correction (one correction-rotation kernel for Q and one
- * for K, skipped when every pair is local), then jl_prefill_attention (the
- * fused tcgen05 attention kernel).
+ *   mode: query shift (jl_qshift) | optional prefill flag (see above).
+ *   workspace: NULL / 0 for the default mode; with JL_PREFILL_FP16 or
+ *   JL_PREFILL_PREROTATED_K device scratch of at least
+ *   jl_prefill_workspace_bytes(...) bytes (contents on entry do not matter;
+ *   overwritten).
+ * Launches: the default mode one kernel (the fused tcgen05 attention kernel,
+ * correcting Q and K itself); the opt-in modes jl_prefill_correction (one or
+ * two correction-rotation kernels) and then the attention kernel.  *dev_error
+ * receives 1 (a pipeline wait ran out) or 3 (a corrected value beyond fp16's
+ * range).
  * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_ALIGNMENT,
  * JL_ERR_WORKSPACE, JL_ERR_CUDA; nothing is launched on an argument error.
  */
@@ -141,13 +166,16 @@ int jl_bifocal_prefill(const void* q, const void* k, const void* v, void* o, flo
 
 /*
  * First stage of jl_bifocal_prefill, exposed so the two stages can be timed or
- * scheduled separately: writes the correction-rotated rows to `workspace`
- * (fp16, [B, L, Hq, D] for R(p_q(i) - i) Q_i followed by [B, L, Hkv, D] for
- * R(f(j) - j) K_j, the second at offset round_up(2 * B * L * Hq * D, 256)).
- * Only rows that have a remote partner are written (queries i >= w0, keys
- * j < L - w0).  The correction identity is the additive composition of RoPE
- * rotations (gist.science summary, "§2 On-the-Fly Correctie Rotatie").
- * Launches nothing when every pair is local.  Errors as jl_bifocal_prefill.
+ * scheduled separately.  Default mode: nothing to do (launches nothing).
+ * JL_PREFILL_FP16: writes R(p_q(i) - i) Q_i as fp16 [B, L, Hq, D] to the
+ * workspace, followed (at offset round_up(2 * B * L * Hq * D, 256)) by
+ * R(f(j) - j) K_j as fp16 [B, L, Hkv, D].  JL_PREFILL_PREROTATED_K: writes the
+ * key rows as fp16 hi [B, L, Hkv, D] and, at offset round_up(2 * B * L * Hkv *
+ * D, 256), lo.  Only rows that have a remote partner are written (queries
+ * i >= w0, keys j < L - w0).  The correction identity is the additive
+ * composition of RoPE rotations (gist.science summary, "§2 On-the-Fly
+ * Correctie Rotatie").  Launches nothing when every pair is local.  Errors as
+ * jl_bifocal_prefill.
  */
 int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, int Hkv, int head_dim, int w0,
                           int w_pretrained, double rope_base, int mode, void* workspace, size_t workspace_bytes,
@@ -155,18 +183,18 @@ int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, in
 
 /*
  * Second stage of jl_bifocal_prefill: the fused tcgen05 attention kernel
- * (one launch), reading Q, K, V and the corrected rows that
- * jl_prefill_correction left in `workspace` (same w0 / w_pretrained / mode).
- * Errors as jl_bifocal_prefill.
+ * (one launch), reading Q, K, V and, in the opt-in modes, the corrected rows
+ * that jl_prefill_correction left in `workspace` (same w0 / w_pretrained /
+ * rope_base / mode).  Errors as jl_bifocal_prefill.
  */
 int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
-                         int Hkv, int head_dim, int w0, int w_pretrained, float softmax_scale, int mode,
-                         const void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
+                         int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,
+                         int mode, const void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
 
 /*
- * Scratch bytes jl_bifocal_prefill_chunk needs: fp16 corrected rows of the
- * chunk's queries [B, chunk_len, Hq, D] and of the keys [B, q_offset +
- * chunk_len, Hkv, D]; twice this with JL_REMOTE_SPLIT.  0 on bad arguments.
+ * Scratch bytes jl_bifocal_prefill_chunk may need in the opt-in modes (as
+ * jl_prefill_workspace_bytes, with chunk_len query rows and q_offset +
+ * chunk_len key rows); the default mode needs none.  0 on bad arguments.
  */
 size_t jl_prefill_chunk_workspace_bytes(int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim);
 
@@ -180,13 +208,13 @@ size_t jl_prefill_chunk_workspace_bytes(int B, int q_offset, int chunk_len, int 
  *   k_cache / v_cache [B, cache_len, Hkv, D]: bf16 device, already holding the
  *   chunk's own keys and values; read only.  q_offset + chunk_len <= cache_len.
  *   o [B, chunk_len, Hq, D] bf16; lse [B, Hq, chunk_len] fp32 or NULL.
- *   workspace: jl_prefill_chunk_workspace_bytes(...) bytes (x2 with
- *   JL_REMOTE_SPLIT).  Everything else as jl_bifocal_prefill.
+ *   workspace: NULL / 0 in the default mode, else
+ *   jl_prefill_chunk_workspace_bytes(...) bytes.  Everything else as
+ *   jl_bifocal_prefill.
  * Note: a cache built by earlier decode steps is not equivalent to re-running
  * prefill over the whole sequence (the keys were rotated once, at their base
  * positions, either way; the hidden states are not recomputed).
- * Launches: two correction kernels (skipped when every pair is local) and the
- * fused attention kernel.
+ * Launches: as jl_bifocal_prefill.
  */
 int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
                              float* lse, int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim, int w0,
@@ -194,8 +222,8 @@ int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_c
                              size_t workspace_bytes, int* dev_error, void* stream);
 
 /*
- * Scratch bytes jl_bifocal_prefill_ie needs (for the given mode): corrected
- * rows for every position, plus three partial outputs and their LSEs.
+ * Scratch bytes jl_bifocal_prefill_ie needs: three fp32 partial outputs
+ * [B, L, Hq, D] and their LSEs [B, Hq, L] (`mode` does not change it).
  */
 size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim, int mode);
 
@@ -204,14 +232,16 @@ size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim
  * per-tile kernel (Jet-Long review, "Method"; gist.science summary, "§2
  * Inclusie-Exclusie Attention Merge"): three attention calls — (A) the window
  * 0 <= i - j < w0 with base RoPE, (B) every causal pair with remote positions,
- * (C) the window with remote positions — each writing a bf16 output and an
- * fp32 LSE, merged as O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C),
- * W_X = exp(LSE_X - max LSE).  Same arguments and result as jl_bifocal_prefill
- * (up to the rounding of the partial outputs, which the subtraction
- * amplifies); workspace: jl_prefill_ie_workspace_bytes(...).  When every pair
- * is local it runs jl_bifocal_prefill.
- * Launches: two correction kernels (all rows), three attention kernels, one
- * merge kernel.
+ * (C) the window with remote positions — each writing an fp32 output and an
+ * fp32 LSE (the default mode's kernel: corrections in the kernel, hi + lo
+ * remote operands; the prefill flags in `mode` are ignored), merged as
+ * O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C), W_X = exp(LSE_X - max
+ * LSE).  Same arguments and result as jl_bifocal_prefill up to rounding, which
+ * the subtraction amplifies by (W_A + W_B + W_C) / (W_A + W_B - W_C): without
+ * bound on rows where one key inside the window dominates both B and C.
+ * workspace: jl_prefill_ie_workspace_bytes(...).  When every pair is local it
+ * runs jl_bifocal_prefill.
+ * Launches: three attention kernels and one merge kernel.
  */
 int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
                           int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,

@@ -383,14 +383,15 @@ def decode_key_range(q, k_cache, v_cache, p: BifocalParams, key_begin: int, key_
 # Second formulation: inclusion-exclusion merge of three masked softmaxes
 # ---------------------------------------------------------------------------
 
-def inclusion_exclusion_rows(q_rows, q_pos, k, v, p: BifocalParams):
-    """The pages' three-call formulation, merged by inclusion-exclusion.
+def inclusion_exclusion_parts(q_rows, q_pos, k, v, p: BifocalParams):
+    """The three calls of the pages' formulation, each a masked softmax.
 
     Jet-Long review, "Method": (A) sliding window with base RoPE, (B) full
-    causal with remote RoPE, (C) sliding window with remote RoPE, merged as
-    O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C) with LSE weights.
-    The window is the local band of ``is_local`` (keys with i - j < w0).
-    Written independently of ``bifocal_scores`` as a cross-check.
+    causal with remote RoPE, (C) sliding window with remote RoPE.  The window
+    is the local band of ``is_local`` (keys with i - j < w0).  Returns
+    ((O_A, LSE_A), (O_B, LSE_B), (O_C, LSE_C)); a row with no key in a call
+    has O = 0, LSE = -inf there.  Written independently of ``bifocal_scores``
+    as a cross-check.
     """
     q_rows = np.asarray(q_rows, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -422,9 +423,17 @@ def inclusion_exclusion_rows(q_rows, q_pos, k, v, p: BifocalParams):
         lse = np.where(ok, msafe + np.log(np.where(ok, l, 1.0)), -np.inf)
         return o, lse
 
-    oa, la = masked(base_s, window)
-    ob, lb = masked(rem_s, causal)
-    oc, lc = masked(rem_s, window)
+    return masked(base_s, window), masked(rem_s, causal), masked(rem_s, window)
+
+
+def inclusion_exclusion_rows(q_rows, q_pos, k, v, p: BifocalParams):
+    """The pages' three-call formulation, merged by inclusion-exclusion.
+
+    Jet-Long review, "Method": the calls of ``inclusion_exclusion_parts``
+    merged as O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C) with LSE
+    weights W_X = exp(LSE_X - max LSE).
+    """
+    (oa, la), (ob, lb), (oc, lc) = inclusion_exclusion_parts(q_rows, q_pos, k, v, p)
     mm = np.maximum(np.maximum(la, lb), lc)
     wa, wb, wc = np.exp(la - mm), np.exp(lb - mm), np.exp(lc - mm)
     den = wa + wb - wc

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libjetlong.so")
-SOURCES = ["jl_api.cu", "rope_rotate.cu", "prefill_sm100.cu", "decode_sm100.cu", "decode_noalloc.cu", "rope_append.cu", "ie_merge.cu"]
+SOURCES = ["jl_api.cu", "rope_rotate.cu", "prefill_sm100.cu", "prefill_hilo_sm100.cu", "decode_sm100.cu", "decode_noalloc.cu", "rope_append.cu", "ie_merge.cu"]
 HEADERS = ["jl_common.cuh", "jl_kernels.cuh", "jl_positions.h", os.path.join("..", "..", "include", "jl_api.h")]
 
 NVCC_FLAGS = [

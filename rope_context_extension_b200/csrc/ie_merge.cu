@@ -7,9 +7,11 @@
 //   LSE = M + ln(W_A + W_B - W_C),  M = max(LSE_A, LSE_B, LSE_C),
 // where A is the window with base RoPE, B every causal pair with remote
 // positions and C the window with remote positions; C removes exactly the part
-// of B that A replaces.  The three partial outputs arrive in bf16, as a
-// FlashAttention call returns them, so the subtraction W_B O_B - W_C O_C sees
-// their rounding.  One warp per (sequence, row, head); memory bound.
+// of B that A replaces.  The three partial outputs arrive in fp32 (the remote
+// calls' scores carry hi + lo operands), so what the subtraction W_B O_B -
+// W_C O_C amplifies is fp32 rounding; where W_B and W_C nearly cancel (a key
+// that dominates both sits in the window) that still grows without bound, a
+// property of the formulation.  One warp per (sequence, row, head).
 #include "jl_kernels.cuh"
 
 namespace jl {
@@ -39,9 +41,9 @@ __global__ void __launch_bounds__(256) ie_merge_kernel(const __grid_constant__ M
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     const int d = lane + 32 * e;
-    const float oa = __bfloat162float(a.o_x[0][obase + d]);
-    const float ob = __bfloat162float(a.o_x[1][obase + d]);
-    const float oc = __bfloat162float(a.o_x[2][obase + d]);
+    const float oa = a.o_x[0][obase + d];
+    const float ob = a.o_x[1][obase + d];
+    const float oc = a.o_x[2][obase + d];
     a.o[obase + d] = __float2bfloat16_rn((wa * oa + wb * ob - wc * oc) * inv);
   }
   if (lane == 0 && a.lse != nullptr) a.lse[lidx] = M + logf(den);

@@ -72,7 +72,8 @@ constexpr int kMaxGridYZ = 65535;  // CUDA's limit on a grid's y and z dimension
 int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained, double rope_base, int mode) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || w0 < 0 || w_pretrained < 1) return JL_ERR_INVALID_ARG;
   if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return JL_ERR_INVALID_ARG;
-  if ((mode & ~(JL_QSHIFT_SELF_EXTEND | JL_REMOTE_SPLIT)) != 0) return JL_ERR_INVALID_ARG;
+  if ((mode & ~(JL_QSHIFT_SELF_EXTEND | JL_PREFILL_FP16 | JL_PREFILL_PREROTATED_K)) != 0) return JL_ERR_INVALID_ARG;
+  if ((mode & JL_PREFILL_FP16) && (mode & JL_PREFILL_PREROTATED_K)) return JL_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
   if (L > (1 << 30)) return JL_ERR_UNSUPPORTED;
@@ -196,15 +197,35 @@ int jl_prefill_tile_classes(int64_t L, int64_t w0, int64_t w_pretrained, int64_t
   return JL_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Prefill scratch (only the opt-in modes use any):
+//   JL_PREFILL_FP16           fp16 corrected query rows [B, Lq, Hq, D], then fp16
+//                             corrected key rows [B, Lk, Hkv, D]
+//   JL_PREFILL_PREROTATED_K   corrected key rows as fp16 hi [B, Lk, Hkv, D], then lo
+// The default mode corrects both sides inside the attention kernel and needs none.
+size_t prefill_ws_fp16(int B, int Lq, int Lk, int Hq, int Hkv, int D) {
+  return round_up((size_t)B * Lq * Hq * D * 2) + round_up((size_t)B * Lk * Hkv * D * 2);
+}
+size_t prefill_ws_prerot(int B, int Lk, int Hkv, int D) { return 2 * round_up((size_t)B * Lk * Hkv * D * 2); }
+size_t prefill_ws_any(int B, int Lq, int Lk, int Hq, int Hkv, int D) {
+  return std::max(prefill_ws_fp16(B, Lq, Lk, Hq, Hkv, D), prefill_ws_prerot(B, Lk, Hkv, D));
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
-  return round_up((size_t)B * L * Hq * head_dim * 2) + round_up((size_t)B * L * Hkv * head_dim * 2);
+  return prefill_ws_any(B, L, L, Hq, Hkv, head_dim);
 }
 
 size_t jl_prefill_chunk_workspace_bytes(int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim) {
   if (B < 1 || q_offset < 0 || chunk_len < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
-  return round_up((size_t)B * chunk_len * Hq * head_dim * 2) +
-         round_up((size_t)B * ((size_t)q_offset + chunk_len) * Hkv * head_dim * 2);
+  return prefill_ws_any(B, chunk_len, q_offset + chunk_len, Hq, Hkv, head_dim);
 }
 
 namespace {
@@ -218,20 +239,32 @@ struct PrefillProblem {
   const void* v;
   int B, q_off, Lq, k_rows, Hq, Hkv, D;
   int Lk() const { return q_off + Lq; }
-  size_t base_ws() const { return jl_prefill_chunk_workspace_bytes(B, q_off, Lq, Hq, Hkv, D); }
 };
 
-__half* q_rem_ptr(void* ws) { return reinterpret_cast<__half*>(ws); }
-__half* k_rem_ptr(void* ws, const PrefillProblem& pp) {
-  return reinterpret_cast<__half*>(reinterpret_cast<char*>(ws) + round_up((size_t)pp.B * pp.Lq * pp.Hq * pp.D * 2));
+bool prefill_all_local(const PrefillProblem& pp, int w0, int w_pretrained) {
+  return jl::all_local(pp.Lk(), w0, jl::group_size(pp.Lk(), w_pretrained));
+}
+
+// Scratch the call needs in this mode (0 for the default mode and whenever
+// every pair is local).
+size_t prefill_ws_need(const PrefillProblem& pp, int w0, int w_pretrained, int mode) {
+  if (prefill_all_local(pp, w0, w_pretrained)) return 0;
+  if (mode & JL_PREFILL_FP16) return prefill_ws_fp16(pp.B, pp.Lq, pp.Lk(), pp.Hq, pp.Hkv, pp.D);
+  if (mode & JL_PREFILL_PREROTATED_K) return prefill_ws_prerot(pp.B, pp.Lk(), pp.Hkv, pp.D);
+  return 0;
+}
+
+__half* ws_first(void* ws) { return reinterpret_cast<__half*>(ws); }
+__half* ws_second(void* ws, size_t first_bytes) {
+  return reinterpret_cast<__half*>(reinterpret_cast<char*>(ws) + round_up(first_bytes));
 }
 
 int problem_checks(const PrefillProblem& pp, int w0, int w_pretrained, double rope_base, int mode) {
   int st = common_checks(pp.B, pp.Lk(), pp.Hq, pp.Hkv, pp.D, w0, w_pretrained, rope_base, mode);
   if (st != JL_OK) return st;
   if (pp.q_off < 0 || pp.Lq < 1 || pp.k_rows < pp.Lk()) return JL_ERR_INVALID_ARG;
-  // attention grid: (query-head groups, 128-row query blocks, batch), with a
-  // 32-bit linear CTA index
+  // attention grid: (query heads or head pairs, 128-row query blocks, batch),
+  // with a 32-bit linear CTA index
   const int64_t blocks = ((int64_t)pp.Lq + 127) / 128;
   if (blocks > kMaxGridYZ || (int64_t)pp.Hq * blocks * pp.B > INT32_MAX) return JL_ERR_UNSUPPORTED;
   if (!pp.q || !pp.k || !pp.v) return JL_ERR_INVALID_ARG;
@@ -241,102 +274,180 @@ int problem_checks(const PrefillProblem& pp, int w0, int w_pretrained, double ro
 
 int workspace_checks(const PrefillProblem& pp, int w0, int w_pretrained, int mode, const void* workspace,
                      size_t workspace_bytes) {
-  const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
-  if (jl::all_local(pp.Lk(), w0, G)) return JL_OK;
-  const size_t need = ((mode & JL_REMOTE_SPLIT) ? 2 : 1) * pp.base_ws();
+  const size_t need = prefill_ws_need(pp, w0, w_pretrained, mode);
+  if (need == 0) return JL_OK;
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
   return JL_OK;
 }
 
+// Correction pass of the opt-in modes (the default mode has none): fp16 rows
+// for JL_PREFILL_FP16, fp16 hi + lo key rows for JL_PREFILL_PREROTATED_K.
 int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double rope_base, int mode,
-                      void* workspace, cudaStream_t s, bool all_rows = false) {
+                      void* workspace, cudaStream_t s) {
+  if (prefill_all_local(pp, w0, w_pretrained)) return JL_OK;  // nothing to correct
+  if (!(mode & (JL_PREFILL_FP16 | JL_PREFILL_PREROTATED_K))) return JL_OK;
   const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
-  if (jl::all_local(pp.Lk(), w0, G)) return JL_OK;  // nothing to correct
-  const bool split = (mode & JL_REMOTE_SPLIT) != 0;
-  char* lo_base = reinterpret_cast<char*>(workspace) + pp.base_ws();  // split: Q_lo then K_lo
   RotateArgs ra;
   std::memset(&ra, 0, sizeof(ra));
   fill_theta(ra.theta, pp.D, rope_base);
   ra.G = G;
   ra.shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
   ra.B = pp.B;
-  // queries that have a remote key: positions q_off + r >= w0
-  ra.x = reinterpret_cast<const __nv_bfloat16*>(pp.q);
-  ra.y = q_rem_ptr(workspace);
-  ra.y_lo = split ? q_rem_ptr(lo_base) : nullptr;
-  ra.x_rows = ra.y_rows = pp.Lq;
-  ra.H = pp.Hq;
-  ra.pos_off = pp.q_off;
-  ra.row_begin = all_rows ? 0 : std::max(0, w0 - pp.q_off);
-  ra.row_end = pp.Lq;
-  ra.is_query = 1;
-  if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
+  const size_t kbytes = (size_t)pp.B * pp.Lk() * pp.Hkv * pp.D * 2;
+  if (mode & JL_PREFILL_FP16) {
+    // queries that have a remote key: positions q_off + r >= w0
+    ra.x = reinterpret_cast<const __nv_bfloat16*>(pp.q);
+    ra.y = ws_first(workspace);
+    ra.y_lo = nullptr;
+    ra.x_rows = ra.y_rows = pp.Lq;
+    ra.H = pp.Hq;
+    ra.pos_off = pp.q_off;
+    ra.row_begin = std::max(0, w0 - pp.q_off);
+    ra.row_end = pp.Lq;
+    ra.is_query = 1;
+    if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
+  }
   // keys that have a remote query: j <= q_off + Lq - 1 - w0
   ra.x = reinterpret_cast<const __nv_bfloat16*>(pp.k);
-  ra.y = k_rem_ptr(workspace, pp);
-  ra.y_lo = split ? k_rem_ptr(lo_base, pp) : nullptr;
+  if (mode & JL_PREFILL_FP16) {
+    ra.y = ws_second(workspace, (size_t)pp.B * pp.Lq * pp.Hq * pp.D * 2);
+    ra.y_lo = nullptr;
+  } else {
+    ra.y = ws_first(workspace);
+    ra.y_lo = ws_second(workspace, kbytes);
+  }
   ra.x_rows = pp.k_rows;
   ra.y_rows = pp.Lk();
   ra.H = pp.Hkv;
   ra.pos_off = 0;
   ra.row_begin = 0;
-  ra.row_end = all_rows ? pp.Lk() : pp.Lk() - w0;
+  ra.row_end = pp.Lk() - w0;
   ra.is_query = 0;
   if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
 
-int attention_launch(const PrefillProblem& pp, void* o, float* lse, int w0, int w_pretrained, float softmax_scale,
-                     int mode, const void* workspace, int* dev_error, cudaStream_t stream, int kind = jl::kBifocal) {
+// Host tables of the in-kernel correction: R(-theta_t b) for b < 16 and
+// R(-theta_t 16 a) for a < 8, formed in fp64 and rounded to fp32.
+void fill_hilo_tables(jl::PrefillHiloArgs& a, int D, double rope_base) {
+  fill_theta(a.theta, D, rope_base);
+  for (int t = 0; t < D / 2; ++t) {
+    for (int b = 0; b < 16; ++b)
+      a.t1[t * 16 + b] = make_float2((float)std::cos(b * a.theta[t]), (float)-std::sin(b * a.theta[t]));
+    for (int m = 0; m < 8; ++m)
+      a.t16[t * 8 + m] = make_float2((float)std::cos(16.0 * m * a.theta[t]), (float)-std::sin(16.0 * m * a.theta[t]));
+  }
+}
+
+// The attention launch.  Every pair local: the two-heads-per-CTA kernel on the
+// bf16 inputs (plain causal RoPE, no rounding of operands).  JL_PREFILL_FP16:
+// the same kernel on the fp16 rows of the correction pass.  Otherwise the hi +
+// lo kernel, correcting Q and K itself (or taking the key rows of
+// JL_PREFILL_PREROTATED_K from the workspace).  o_f32 (inclusion-exclusion
+// partials) writes fp32 instead of bf16 output.
+int attention_launch(const PrefillProblem& pp, void* o, float* o_f32, float* lse, int w0, int w_pretrained,
+                     double rope_base, float softmax_scale, int mode, const void* workspace, int* dev_error,
+                     cudaStream_t stream, int kind = jl::kBifocal) {
   const int D = pp.D;
   const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
   const bool all_local = kind == jl::kBifocal && jl::all_local(pp.Lk(), w0, G);
-  const bool split = !all_local && (mode & JL_REMOTE_SPLIT) != 0;
-  CUtensorMap tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo;
-  if (!encode_bf16_4d(&tq, pp.q, D, pp.Hq, pp.Lq, pp.B, 128) ||
-      !encode_bf16_4d(&tk, pp.k, D, pp.Hkv, pp.k_rows, pp.B, 128) ||
+  const int r = pp.Hq / pp.Hkv;
+  const float scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
+  CUtensorMap tk, tv;
+  if (!encode_bf16_4d(&tk, pp.k, D, pp.Hkv, pp.k_rows, pp.B, 128) ||
       !encode_bf16_4d(&tv, pp.v, D, pp.Hkv, pp.k_rows, pp.B, 128))
     return JL_ERR_CUDA;
-  if (!all_local) {
+  if (all_local || (mode & JL_PREFILL_FP16)) {
+    if (kind != jl::kBifocal || o_f32 != nullptr) return JL_ERR_INVALID_ARG;
+    CUtensorMap tq, tqr, tkr;
+    if (!encode_bf16_4d(&tq, pp.q, D, pp.Hq, pp.Lq, pp.B, 128)) return JL_ERR_CUDA;
+    if (!all_local) {
+      void* ws = const_cast<void*>(workspace);
+      if (!encode_f16_4d(&tqr, ws_first(ws), D, pp.Hq, pp.Lq, pp.B, 128) ||
+          !encode_f16_4d(&tkr, ws_second(ws, (size_t)pp.B * pp.Lq * pp.Hq * pp.D * 2), D, pp.Hkv, pp.Lk(), pp.B,
+                         128))
+        return JL_ERR_CUDA;
+    } else {
+      tqr = tq;
+      tkr = tk;
+    }
+    PrefillArgs pa;
+    std::memset(&pa, 0, sizeof(pa));
+    pa.o = reinterpret_cast<__nv_bfloat16*>(o);
+    pa.lse = lse;
+    pa.dev_error = dev_error;
+    pa.B = pp.B;
+    pa.Hq = pp.Hq;
+    pa.Hkv = pp.Hkv;
+    pa.r = r;
+    pa.q_off = pp.q_off;
+    pa.Lq = pp.Lq;
+    pa.Lk = pp.Lk();
+    pa.nh = r % 2 == 0 ? 2 : 1;
+    pa.num_mb = (pp.Lq + 127) / 128;
+    pa.all_local = all_local ? 1 : 0;
+    pa.w0 = all_local ? (1 << 30) : w0;
+    pa.scale_log2 = scale_log2;
+    if (jl::launch_prefill(tq, tqr, tk, tkr, tv, pa, D, stream) != cudaSuccess) return JL_ERR_CUDA;
+    return JL_OK;
+  }
+  const bool rot_k = !(mode & JL_PREFILL_PREROTATED_K);
+  CUtensorMap tkh = tk, tkl = tk;
+  if (!rot_k) {
     void* ws = const_cast<void*>(workspace);
-    if (!encode_f16_4d(&tqr, q_rem_ptr(ws), D, pp.Hq, pp.Lq, pp.B, 128) ||
-        !encode_f16_4d(&tkr, k_rem_ptr(ws, pp), D, pp.Hkv, pp.Lk(), pp.B, 128))
+    const size_t kbytes = (size_t)pp.B * pp.Lk() * pp.Hkv * pp.D * 2;
+    if (!encode_f16_4d(&tkh, ws_first(ws), D, pp.Hkv, pp.Lk(), pp.B, 128) ||
+        !encode_f16_4d(&tkl, ws_second(ws, kbytes), D, pp.Hkv, pp.Lk(), pp.B, 128))
       return JL_ERR_CUDA;
-  } else {
-    tqr = tq;
-    tkr = tk;
   }
-  if (split) {
-    void* lo = reinterpret_cast<char*>(const_cast<void*>(workspace)) + pp.base_ws();
-    if (!encode_f16_4d(&tqr_lo, q_rem_ptr(lo), D, pp.Hq, pp.Lq, pp.B, 128) ||
-        !encode_f16_4d(&tkr_lo, k_rem_ptr(lo, pp), D, pp.Hkv, pp.Lk(), pp.B, 128))
-      return JL_ERR_CUDA;
-  } else {
-    tqr_lo = tqr;
-    tkr_lo = tkr;
+  static_assert(sizeof(jl::PrefillHiloArgs) + 4 * sizeof(CUtensorMap) <= 32764, "kernel parameters too large");
+  jl::PrefillHiloArgs ha;
+  std::memset(&ha, 0, sizeof(ha));
+  ha.q = reinterpret_cast<const __nv_bfloat16*>(pp.q);
+  ha.k = reinterpret_cast<const __nv_bfloat16*>(pp.k);
+  ha.o = reinterpret_cast<__nv_bfloat16*>(o);
+  ha.o_f32 = o_f32;
+  ha.lse = lse;
+  ha.dev_error = dev_error;
+  ha.B = pp.B;
+  ha.Hq = pp.Hq;
+  ha.Hkv = pp.Hkv;
+  ha.r = r;
+  ha.q_off = pp.q_off;
+  ha.Lq = pp.Lq;
+  ha.k_rows = pp.k_rows;
+  ha.num_mb = (pp.Lq + 127) / 128;
+  ha.w0 = w0;
+  ha.kind = kind;
+  ha.G = G;
+  ha.shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
+  ha.scale_log2 = scale_log2;
+  fill_hilo_tables(ha, D, rope_base);
+  if (jl::launch_prefill_hilo(tk, tv, tkh, tkl, ha, D, rot_k, stream) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int prefill_entry(const PrefillProblem& pp, void* o, float* lse, int w0, int w_pretrained, double rope_base,
+                  float softmax_scale, int mode, void* workspace, size_t workspace_bytes, int* dev_error,
+                  void* stream, bool correct, bool attend) {
+  // Validate everything before the first launch.
+  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
+  if (st != JL_OK) return st;
+  if (attend) {
+    if (!o) return JL_ERR_INVALID_ARG;
+    if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
   }
-  const int r = pp.Hq / pp.Hkv;
-  PrefillArgs pa;
-  std::memset(&pa, 0, sizeof(pa));
-  pa.o = reinterpret_cast<__nv_bfloat16*>(o);
-  pa.lse = lse;
-  pa.dev_error = dev_error;
-  pa.B = pp.B;
-  pa.Hq = pp.Hq;
-  pa.Hkv = pp.Hkv;
-  pa.r = r;
-  pa.q_off = pp.q_off;
-  pa.Lq = pp.Lq;
-  pa.Lk = pp.Lk();
-  pa.nh = (!split && r % 2 == 0) ? 2 : 1;
-  pa.num_mb = (pp.Lq + 127) / 128;
-  pa.all_local = all_local ? 1 : 0;
-  pa.w0 = all_local ? (1 << 30) : w0;
-  pa.kind = kind;
-  pa.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
-  if (jl::launch_prefill(tq, tqr, tk, tkr, tv, tqr_lo, tkr_lo, pa, D, split, stream) != cudaSuccess)
-    return JL_ERR_CUDA;
+  st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
+  if (st != JL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (correct) {
+    st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s);
+    if (st != JL_OK) return st;
+  }
+  if (attend)
+    return attention_launch(pp, o, nullptr, lse, w0, w_pretrained, rope_base, softmax_scale, mode, workspace,
+                            dev_error, s);
   return JL_OK;
 }
 
@@ -346,41 +457,24 @@ int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, in
                           int w_pretrained, double rope_base, int mode, void* workspace, size_t workspace_bytes,
                           void* stream) {
   const PrefillProblem pp{q, k, k, B, 0, L, L, Hq, Hkv, head_dim};
-  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
-  if (st == JL_OK) st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
-  if (st != JL_OK) return st;
-  return correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, reinterpret_cast<cudaStream_t>(stream));
+  return prefill_entry(pp, nullptr, nullptr, w0, w_pretrained, rope_base, 0.f, mode, workspace, workspace_bytes,
+                       nullptr, stream, true, false);
 }
 
 int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
-                         int Hkv, int head_dim, int w0, int w_pretrained, float softmax_scale, int mode,
-                         const void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
+                         int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,
+                         int mode, const void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
   const PrefillProblem pp{q, k, v, B, 0, L, L, Hq, Hkv, head_dim};
-  int st = problem_checks(pp, w0, w_pretrained, 10000.0, mode);
-  if (st != JL_OK) return st;
-  if (!o) return JL_ERR_INVALID_ARG;
-  if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
-  st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
-  if (st != JL_OK) return st;
-  return attention_launch(pp, o, lse, w0, w_pretrained, softmax_scale, mode, workspace, dev_error,
-                          reinterpret_cast<cudaStream_t>(stream));
+  return prefill_entry(pp, o, lse, w0, w_pretrained, rope_base, softmax_scale, mode, const_cast<void*>(workspace),
+                       workspace_bytes, dev_error, stream, false, true);
 }
 
 int jl_bifocal_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
                        int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,
                        int mode, void* workspace, size_t workspace_bytes, int* dev_error, void* stream) {
-  // Validate everything before the first launch.
   const PrefillProblem pp{q, k, v, B, 0, L, L, Hq, Hkv, head_dim};
-  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
-  if (st != JL_OK) return st;
-  if (!o) return JL_ERR_INVALID_ARG;
-  if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
-  st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
-  if (st != JL_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s);
-  if (st != JL_OK) return st;
-  return attention_launch(pp, o, lse, w0, w_pretrained, softmax_scale, mode, workspace, dev_error, s);
+  return prefill_entry(pp, o, lse, w0, w_pretrained, rope_base, softmax_scale, mode, workspace, workspace_bytes,
+                       dev_error, stream, true, true);
 }
 
 int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_cache, int64_t cache_len, void* o,
@@ -390,16 +484,8 @@ int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_c
   if (cache_len < 1 || cache_len > ((int64_t)1 << 30)) return JL_ERR_INVALID_ARG;
   if (q_offset < 0 || chunk_len < 1 || (int64_t)q_offset + chunk_len > cache_len) return JL_ERR_INVALID_ARG;
   const PrefillProblem pp{q, k_cache, v_cache, B, q_offset, chunk_len, (int)cache_len, Hq, Hkv, head_dim};
-  int st = problem_checks(pp, w0, w_pretrained, rope_base, mode);
-  if (st != JL_OK) return st;
-  if (!o) return JL_ERR_INVALID_ARG;
-  if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
-  st = workspace_checks(pp, w0, w_pretrained, mode, workspace, workspace_bytes);
-  if (st != JL_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s);
-  if (st != JL_OK) return st;
-  return attention_launch(pp, o, lse, w0, w_pretrained, softmax_scale, mode, workspace, dev_error, s);
+  return prefill_entry(pp, o, lse, w0, w_pretrained, rope_base, softmax_scale, mode, workspace, workspace_bytes,
+                       dev_error, stream, true, true);
 }
 
 namespace {
@@ -407,12 +493,12 @@ namespace {
 struct IeLayout {
   size_t o[3], lse[3], total;
 };
-IeLayout ie_layout(int B, int L, int Hq, int Hkv, int D, int mode) {
+IeLayout ie_layout(int B, int L, int Hq, int D) {
   IeLayout lay;
-  size_t off = ((mode & JL_REMOTE_SPLIT) ? 2 : 1) * jl_prefill_workspace_bytes(B, L, Hq, Hkv, D);
+  size_t off = 0;
   for (int x = 0; x < 3; ++x) {
     lay.o[x] = off;
-    off += round_up((size_t)B * L * Hq * D * 2);
+    off += round_up((size_t)B * L * Hq * D * 4);
   }
   for (int x = 0; x < 3; ++x) {
     lay.lse[x] = off;
@@ -425,8 +511,9 @@ IeLayout ie_layout(int B, int L, int Hq, int Hkv, int D, int mode) {
 }  // namespace
 
 size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim, int mode) {
+  (void)mode;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
-  return ie_layout(B, L, Hq, Hkv, head_dim, mode).total;
+  return ie_layout(B, L, Hq, head_dim).total;
 }
 
 int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
@@ -437,29 +524,28 @@ int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, 
   if (st != JL_OK) return st;
   if (!o) return JL_ERR_INVALID_ARG;
   if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
+  const int qmode = mode & JL_QSHIFT_SELF_EXTEND;  // the three calls always correct in the kernel, hi + lo
   const int64_t G = jl::group_size(L, w_pretrained);
   if (jl::all_local(L, w0, G)) {
     // every pair local: the three calls collapse to plain causal attention
     return jl_bifocal_prefill(q, k, v, o, lse, B, L, Hq, Hkv, head_dim, w0, w_pretrained, rope_base, softmax_scale,
-                              mode, workspace, workspace_bytes, dev_error, stream);
+                              qmode, nullptr, 0, dev_error, stream);
   }
-  const IeLayout lay = ie_layout(B, L, Hq, Hkv, head_dim, mode);
+  const IeLayout lay = ie_layout(B, L, Hq, head_dim);
   if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* ws = reinterpret_cast<char*>(workspace);
-  // call B scores every causal pair with corrected rows: correct all rows
-  st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s, /*all_rows=*/true);
-  if (st != JL_OK) return st;
   const int kinds[3] = {jl::kWindowBase, jl::kCausalRemote, jl::kWindowRemote};
   jl::MergeArgs ma;
   std::memset(&ma, 0, sizeof(ma));
   for (int x = 0; x < 3; ++x) {
-    void* ox = ws + lay.o[x];
+    float* ox = reinterpret_cast<float*>(ws + lay.o[x]);
     float* lx = reinterpret_cast<float*>(ws + lay.lse[x]);
-    st = attention_launch(pp, ox, lx, w0, w_pretrained, softmax_scale, mode, workspace, dev_error, s, kinds[x]);
+    st = attention_launch(pp, nullptr, ox, lx, w0, w_pretrained, rope_base, softmax_scale, qmode, nullptr, dev_error,
+                          s, kinds[x]);
     if (st != JL_OK) return st;
-    ma.o_x[x] = reinterpret_cast<const __nv_bfloat16*>(ox);
+    ma.o_x[x] = ox;
     ma.lse_x[x] = lx;
   }
   ma.o = reinterpret_cast<__nv_bfloat16*>(o);

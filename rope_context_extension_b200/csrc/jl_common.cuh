@@ -17,6 +17,7 @@ namespace jl {
 enum : int {
   kDevOk = 0,
   kDevTimeout = 1,  // a bounded mbarrier wait ran out; results are invalid
+  kDevRange = 3,    // a corrected query / key value is beyond fp16's range; results are invalid
 };
 
 // A wait that has not completed after this long means the pipeline is stuck.

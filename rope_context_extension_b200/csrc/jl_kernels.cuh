@@ -23,7 +23,8 @@ struct RotateArgs {
 };
 cudaError_t launch_rotate_rows(const RotateArgs& args, int D, cudaStream_t stream);
 
-// Fused bifocal prefill (tcgen05 + TMEM + TMA).
+// Fused bifocal prefill from fp16 corrected rows (tcgen05 + TMEM + TMA; two
+// query heads per CTA).
 struct PrefillArgs {
   __nv_bfloat16* o;  // [B, Lq, Hq, D]
   float* lse;        // [B, Hq, Lq] or null
@@ -36,13 +37,39 @@ struct PrefillArgs {
   int num_mb;        // ceil(Lq / 128)
   int w0;            // band width; huge when every pair is local
   int all_local;
-  int kind;          // kBifocal, or one call of the inclusion-exclusion formulation
   float scale_log2;  // softmax scale * log2(e)
 };
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
-                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
-                           const CUtensorMap& tm_kr_lo, const PrefillArgs& a, int D, bool split,
+                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const PrefillArgs& a, int D,
                            cudaStream_t stream);
+
+// Fused bifocal prefill with the correction rotation inside the kernel and
+// remote scores from fp16 hi + lo operands (tcgen05 + TMEM; one query head per
+// CTA).  With rot_k = false the key tiles' hi / lo rows come from the
+// correction pass through tm_kh / tm_kl instead of being rotated in the kernel.
+struct PrefillHiloArgs {
+  const __nv_bfloat16* q;  // [B, Lq, Hq, D], rotated at the absolute positions
+  const __nv_bfloat16* k;  // [B, k_rows, Hkv, D]
+  __nv_bfloat16* o;        // [B, Lq, Hq, D] bf16 output (when o_f32 is null)
+  float* o_f32;            // [B, Lq, Hq, D] fp32 output instead (inclusion-exclusion partials), or null
+  float* lse;              // [B, Hq, Lq] or null
+  int* dev_error;          // device int or null
+  int B, Hq, Hkv, r;
+  int q_off;               // position of query row 0
+  int Lq;                  // query rows (this chunk)
+  int k_rows;              // rows of K / V
+  int num_mb;              // ceil(Lq / 128)
+  int w0;
+  int kind;                // kBifocal, or one call of the inclusion-exclusion formulation
+  int64_t G, shift;        // group size and query shift (from the total length q_off + Lq)
+  float scale_log2;        // softmax scale * log2(e)
+  double theta[kMaxHalfDim];
+  float2 t1[kMaxHalfDim * 16];   // R(-theta_t b) for b < 16, [t][b] (cos, sin)
+  float2 t16[kMaxHalfDim * 8];   // R(-theta_t 16 a) for a < 8, [t][a]
+};
+cudaError_t launch_prefill_hilo(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_kh,
+                                const CUtensorMap& tm_kl, const PrefillHiloArgs& a, int D, bool rot_k,
+                                cudaStream_t stream);
 
 // Split-KV bifocal decode (mma.sync tiles, in-register correction of keys).
 struct DecodeArgs {
@@ -85,7 +112,7 @@ int decode_in_fixed_scratch(const void* q, const void* k_cache, const void* v_ca
 
 // Inclusion-exclusion merge of three partial prefill outputs.
 struct MergeArgs {
-  const __nv_bfloat16* o_x[3];  // O_A, O_B, O_C [B, L, Hq, D]
+  const float* o_x[3];          // O_A, O_B, O_C [B, L, Hq, D] (fp32)
   const float* lse_x[3];        // LSE_A, LSE_B, LSE_C [B, Hq, L] (natural log)
   __nv_bfloat16* o;
   float* lse;                   // or null

@@ -1,0 +1,777 @@
+// Fused Dynamic Bifocal RoPE prefill for sm_100a, with the correction rotation
+// applied inside the kernel and remote scores carried at about 22 significant
+// bits.
+//
+// A causal (query i, key j) pair with i - j < w0 is scored with the base-rotated
+// Q and K (exact base RoPE); every other causal pair with R(p_q(i)) q and
+// R(f(j)) k (Jet-Long review, "Method"; gist.science summary, "Methodologie
+// §1").  The inputs are rotated at their absolute positions, so the remote rows
+// are R(dq_i) Q_i and R(dk_j) K_j with dq_i = p_q(i) - i, dk_j = f(j) - j: RoPE
+// rotations compose additively (gist.science summary, "§2 On-the-Fly Correctie
+// Rotatie").  Nothing is written back to the inputs or to any scratch buffer:
+//   * a rotation warpgroup reads each key row of a remote tile from global
+//     memory one tile ahead, rotates it in fp32 registers and writes it into
+//     shared memory as fp16 hi + lo (hi = fp16(x), lo = fp16(x - hi)), in the
+//     128-byte-swizzled K-major layout the tensor core reads;
+//   * the same warpgroup rotates the block's query rows once into TMEM
+//     (Q_hi and Q_lo, the A operands);
+//   * a remote score tile is S = Q_hi K_hi + Q_hi K_lo + Q_lo K_hi (fp32
+//     accumulate): the operands carry about 22 significant bits, so a score's
+//     rounding error is about 2^-21 of |q| |k| instead of 2^-11 for one fp16
+//     product (which is what a key of large norm that dominates a softmax row
+//     turns into an LSE error).
+// Correction angles theta_t * dk come from a per-tile factor R(theta_t (dk_j0 -
+// 16 a)) (fp64 sincos, one per (tile, t), times a fixed table) and a 16-entry
+// table R(-theta_t b), with dk_j = dk_j0 - (16 a + b) inside the tile.
+//
+// Each 128 x 128 (query block, key block) tile is visited once per score set it
+// needs (remote passes first, then local passes; a tile straddling the band
+// edge gets both, with complementary masks), all feeding one online softmax.
+//
+// CTA = one 128-row query block of one query head.  Warp roles (384 threads):
+//   warp 0      TMA producer: V (2 stages); K (pre-rotated variant only)
+//   warp 1      tcgen05 MMA issuer; owns the TMEM allocation (512 columns)
+//   warps 4-7   softmax (thread = query row = TMEM lane)
+//   warps 8-11  rotation: query rows into TMEM, key tiles into shared memory
+// TMEM columns: S double buffer at 0 / 128 (P, bf16, overwrites the first 64
+// columns of its S), O at 256, Q_hi (or the base Q) at 256 + D, Q_lo at
+// 256 + 3D/2.  MMA order S(0) S(1) PV(0) S(2) PV(1) S(3) ...: the tensor core
+// computes the next tile's scores while the softmax works on this one.
+#include "jl_kernels.cuh"
+
+namespace jl {
+
+namespace {
+
+constexpr int kHThreads = 384;
+constexpr int kHStages = 2;
+constexpr int kHLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
+constexpr int kHLowRegs = 104;     // warpgroup 0: TMA producer, MMA issuer
+constexpr int kHHighRegs = 200;    // warpgroups 1-2: softmax, rotation
+static_assert(128 * kHLowRegs + 256 * kHHighRegs <= kHThreads * kHLaunchRegs, "register split exceeds the launch pool");
+constexpr int kSlab = 128 * 128;  // one 128-row x 128-byte swizzled slab
+
+template <int D>
+struct HCfg {
+  static constexpr int kChunks = D / 64;  // 64-element (128 B) slabs per row
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kKOff = 0;                               // [stage][hi | lo]
+  static constexpr int kVOff = kKOff + kHStages * 2 * kTile;    // [stage]
+  static constexpr int kT1Off = kVOff + kHStages * kTile;       // R(-theta_t b): [t/2][b][t&1] float2
+  static constexpr int kT1Bytes = (D / 2) * 16 * 8;
+  static constexpr int kCOff = kT1Off + kT1Bytes;               // [buffer][t/2][a][t&1] float2
+  static constexpr int kCBytes = (D / 2) * 8 * 8;               // buffers 0, 1: key tiles; 2: query block
+  static constexpr int kBarOff = kCOff + 3 * kCBytes;
+  static constexpr int kUsed = kBarOff + 256;
+  // At least 120 KB so only one CTA is resident per SM (each allocates 512
+  // TMEM columns).
+  static constexpr int kSmem = (kUsed < 120 * 1024 ? 120 * 1024 : kUsed) + 1024;
+};
+
+// barrier slots
+enum {
+  hKFull = 0,         // [stage]: rotated (or copied) key tile in shared memory
+  hKEmpty = 2,        // [stage]: the score products reading it have completed
+  hVFull = 4,
+  hVEmpty = 6,
+  hSFull = 8,         // [S buffer]
+  hPFull = 10,        // [S buffer][64-key half of P]
+  hPVDone = 14,       // O += P V of the latest pass has completed
+  hQReady = 16,       // the query operands are in TMEM (phase 0: first pass kind, 1: after the switch)
+  hQEmpty = 17,       // the last product reading the first query operands has completed
+  hCReady = 18,       // rotation warpgroup: factor table of the next tile written
+  hOFinal = 19,
+  hDrain = 20,
+  hNumBars = 21
+};
+static_assert(hNumBars * 8 <= 192, "barrier block overflow");
+
+__device__ __forceinline__ bool h_drain_wait(uint32_t bar, uint32_t parity) {
+  // Only after an abort: wait (up to ~100 ms) for async work already in flight
+  // so the CTA never exits while a copy or an MMA still targets it.
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > 100000000ull) return false;
+  }
+  return true;
+}
+
+struct HPass {
+  int nb;       // key block
+  bool remote;  // corrected operands (hi + lo) or base operands
+  int mask;     // 0: band 0 <= i-j < w0, 1: beyond the band i-j >= w0, 2: every causal pair
+};
+
+// Pass p of a query block: the fused method visits its remote passes first
+// (key blocks nb_rem_max .. 0), then its local passes (nb_max down); the
+// inclusion-exclusion calls visit one kind only.
+template <int kind>
+__device__ __forceinline__ HPass hilo_pass(const Sched& s, int p) {
+  HPass r;
+  if (kind == kBifocal) {
+    if (p < s.n_rem) {
+      r.nb = s.nb_rem_max - p;
+      r.remote = true;
+      r.mask = 1;
+    } else {
+      r.nb = s.nb_max - (p - s.n_rem);
+      r.remote = false;
+      r.mask = 0;
+    }
+  } else {
+    r.nb = s.nb_max - p;
+    r.remote = kind != kWindowBase;
+    r.mask = kind == kCausalRemote ? 2 : 0;
+  }
+  return r;
+}
+
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// x rounded to fp16 (hi) and the rounding residual rounded to fp16 (lo), for
+// two values; hi + lo carries about 22 significant bits.
+__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Bit 15 / 31 of the result is set when that fp16 half of h is inf or NaN.
+__device__ __forceinline__ uint32_t f16x2_nonfinite_bits(uint32_t h) { return (h & 0x7FFF7FFFu) + 0x04000400u; }
+
+// Rotates one row of D bf16 values (half-split pairs (t, t + D/2), D/2 words of
+// two consecutive dims each) by R(theta_t (base - delta)) with the factor
+// C[t][delta >> 4] * T1[t][delta & 15] (C = R(theta_t (base - 16 a)), T1 =
+// R(-theta_t b)), and hands each 8-dim unit U (flat index over the row) of the
+// fp16 hi and lo results to emit(U, hi[4], lo[4]).  Non-finite hi halves are
+// recorded in *range.
+template <int D, typename Emit>
+__device__ __forceinline__ void rotate_row_hilo(const uint32_t (&raw)[D / 2], const float2* Cb, const float2* T1s,
+                                                int delta, uint32_t& range, Emit&& emit) {
+  constexpr int H2 = D / 2;
+  const int a = delta >> 4, bb = delta & 15;
+#pragma unroll
+  for (int u = 0; u < H2 / 8; ++u) {
+    uint32_t hx[4], lx[4], hy[4], ly[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = 8 * u + 2 * k;
+      const float4 cf = *reinterpret_cast<const float4*>(&Cb[((t >> 1) * 8 + a) * 2]);
+      const float4 tf = *reinterpret_cast<const float4*>(&T1s[((t >> 1) * 16 + bb) * 2]);
+      const float c0 = cf.x * tf.x - cf.y * tf.y, s0 = cf.x * tf.y + cf.y * tf.x;
+      const float c1 = cf.z * tf.z - cf.w * tf.w, s1 = cf.z * tf.w + cf.w * tf.z;
+      const uint32_t xw = raw[t / 2], yw = raw[(t + H2) / 2];
+      const float x0 = bf16lo_to_f32(xw), x1 = bf16hi_to_f32(xw);
+      const float y0 = bf16lo_to_f32(yw), y1 = bf16hi_to_f32(yw);
+      // (x, y) -> (x cos - y sin, y cos + x sin)
+      split_f16x2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1, hx[k], lx[k]);
+      split_f16x2(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1, hy[k], ly[k]);
+      range |= f16x2_nonfinite_bits(hx[k]) | f16x2_nonfinite_bits(hy[k]);
+    }
+    emit(u, hx, lx);
+    emit(u + H2 / 8, hy, ly);
+  }
+}
+
+template <int D, bool kRotK, int kKind>
+__global__ void __launch_bounds__(kHThreads, 1)
+    bifocal_prefill_hilo_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                                const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kl,
+                                const __grid_constant__ PrefillHiloArgs args) {
+  using C = HCfg<D>;
+  constexpr int H2 = D / 2;
+  constexpr uint32_t kColO = 256, kColQA = 256 + D, kColQB = 256 + D + D / 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 196);
+  auto bar = [&](int i) -> uint32_t { return smem_addr(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Work order (CTAs launch in increasing linear index): the CTAs of one KV
+  // head's query heads run together, heaviest query blocks first, so the CTAs
+  // resident at any time read the same K / V rows and find them in L2.
+  const int r = args.r;
+  int lin = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+  const int hg = lin % r;
+  lin /= r;
+  const int mb = args.num_mb - 1 - lin % args.num_mb;
+  lin /= args.num_mb;
+  const int kvh = lin % args.Hkv;
+  const int b = lin / args.Hkv;
+  const int hq = kvh * r + hg;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kHStages; ++s) {
+      mbar_init(bar(hKFull + s), kRotK ? 128 : 1);
+      mbar_init(bar(hKEmpty + s), 1);
+      mbar_init(bar(hVFull + s), 1);
+      mbar_init(bar(hVEmpty + s), 1);
+      mbar_init(bar(hSFull + s), 1);
+      mbar_init(bar(hPFull + 2 * s), 128);
+      mbar_init(bar(hPFull + 2 * s + 1), 128);
+    }
+    mbar_init(bar(hPVDone), 1);
+    mbar_init(bar(hQReady), 128);
+    mbar_init(bar(hQEmpty), 1);
+    mbar_init(bar(hCReady), 128);
+    mbar_init(bar(hOFinal), 1);
+    mbar_init(bar(hDrain), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), 512u);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int off = args.q_off + mb * 128;                             // position of this block's first query
+  const int last = min(off + 127, args.q_off + args.Lq - 1);         // its last query row
+  const Sched sc = make_sched<kKind>(off, last, args.w0, false);
+  const int npass = sc.n_loc + sc.n_rem;
+  const bool q_switch = kKind == kBifocal && sc.n_loc > 0 && sc.n_rem > 0;
+  const int p_switch = sc.n_rem;  // first local pass (fused method)
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHLowRegs));
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ producer
+      tma_prefetch_map(&tm_v);
+      if (!kRotK) {
+        tma_prefetch_map(&tm_k);
+        tma_prefetch_map(&tm_kh);
+        tma_prefetch_map(&tm_kl);
+      }
+      int k_last = -1, v_last = -1;
+      bool ok = true;
+      for (int p = 0; p < npass; ++p) {
+        const int s = p & 1;
+        const uint32_t ph = (uint32_t)(p >> 1) & 1u;
+        const HPass ps = hilo_pass<kKind>(sc, p);
+        if (!kRotK) {
+          if (!(ok = mbar_wait(bar(hKEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
+          const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
+          mbar_arrive_expect_tx(bar(hKFull + s), (uint32_t)((ps.remote ? 2 : 1) * C::kTile));
+          for (int c = 0; c < C::kChunks; ++c) {
+            if (ps.remote) {
+              tma_load_4d(khi + c * kSlab, &tm_kh, bar(hKFull + s), c * 64, kvh, ps.nb * 128, b);
+              tma_load_4d(khi + C::kTile + c * kSlab, &tm_kl, bar(hKFull + s), c * 64, kvh, ps.nb * 128, b);
+            } else {
+              tma_load_4d(khi + c * kSlab, &tm_k, bar(hKFull + s), c * 64, kvh, ps.nb * 128, b);
+            }
+          }
+          k_last = p;
+        }
+        if (!(ok = mbar_wait(bar(hVEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
+        mbar_arrive_expect_tx(bar(hVFull + s), (uint32_t)C::kTile);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sbase + C::kVOff + s * C::kTile + c * kSlab, &tm_v, bar(hVFull + s), c * 64, kvh,
+                      ps.nb * 128, b);
+        v_last = p;
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA can exit.
+        for (int p = max(0, k_last - kHStages + 1); p <= k_last; ++p)
+          h_drain_wait(bar(hKFull + (p & 1)), (uint32_t)(p >> 1) & 1u);
+        for (int p = max(0, v_last - kHStages + 1); p <= v_last; ++p)
+          h_drain_wait(bar(hVFull + (p & 1)), (uint32_t)(p >> 1) & 1u);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t id_loc = make_idesc_16bit(128, 128, false, false);  // bf16 Q K
+      const uint32_t id_rem = make_idesc_16bit(128, 128, false, true);   // fp16 Q_hi / Q_lo, K_hi / K_lo
+      const uint32_t id_pv = make_idesc_16bit(128, D, true, false);      // bf16 P V
+      auto issue_s = [&](int p) -> bool {
+        const int s = p & 1;
+        const uint32_t ph = (uint32_t)(p >> 1) & 1u;
+        if (p == 0 || (q_switch && p == p_switch)) {
+          if (!mbar_wait(bar(hQReady), p == 0 ? 0u : 1u, abort_flag, args.dev_error)) return false;
+        }
+        if (!mbar_wait(bar(hKFull + s), ph, abort_flag, args.dev_error)) return false;
+        tc_fence_after();
+        const HPass ps = hilo_pass<kKind>(sc, p);
+        const uint32_t d = tmem + (uint32_t)(128 * s);
+        const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
+        const uint32_t klo = khi + C::kTile;
+        const uint32_t id_s = ps.remote ? id_rem : id_loc;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t o = (uint32_t)((ks >> 2) * kSlab + (ks & 3) * 32);
+          mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), make_sdesc_sw128(khi + o, 16, 1024), id_s, ks > 0 ? 1u : 0u);
+        }
+        if (ps.remote) {
+          // + Q_hi K_lo + Q_lo K_hi into the same accumulator
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t o = (uint32_t)((ks >> 2) * kSlab + (ks & 3) * 32);
+            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), make_sdesc_sw128(klo + o, 16, 1024), id_s, 1u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t o = (uint32_t)((ks >> 2) * kSlab + (ks & 3) * 32);
+            mma_ts(d, tmem + kColQB + (uint32_t)(ks * 8), make_sdesc_sw128(khi + o, 16, 1024), id_s, 1u);
+          }
+        }
+        tc_commit(bar(hSFull + s));
+        tc_commit(bar(hKEmpty + s));
+        if (q_switch && p == p_switch - 1) tc_commit(bar(hQEmpty));
+        return true;
+      };
+      // O += P V in two 64-key halves, each issued as soon as the softmax has
+      // written that half of P.
+      auto issue_pv = [&](int p) -> bool {
+        const int s = p & 1;
+        const uint32_t ph = (uint32_t)(p >> 1) & 1u;
+        if (!mbar_wait(bar(hVFull + s), ph, abort_flag, args.dev_error)) return false;
+        const uint32_t va = sbase + C::kVOff + s * C::kTile;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(bar(hPFull + 2 * s + half), ph, abort_flag, args.dev_error)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int ks = half * 4 + kk;
+            // V is MN-major here: 64-dim slabs kSlab apart, 8-key groups 1024 B apart.
+            mma_ts(tmem + kColO, tmem + (uint32_t)(128 * s + ks * 8),
+                   make_sdesc_sw128(va + (uint32_t)(ks * 2048), kSlab, 1024), id_pv, (p > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(bar(hVEmpty + s));
+        tc_commit(bar(hPVDone));
+        return true;
+      };
+      bool ok = true;
+      if (npass > 0) {
+        ok = issue_s(0);
+        if (ok && npass > 1) ok = issue_s(1);
+        for (int p = 0; p < npass && ok; ++p) {
+          ok = issue_pv(p);
+          if (ok && p + 2 < npass) ok = issue_s(p + 2);
+        }
+      }
+      // Every product issued must have completed before TMEM is released.
+      if (ok) {
+        tc_commit(bar(hOFinal));
+        h_drain_wait(bar(hOFinal), 0);
+      } else {
+        tc_commit(bar(hDrain));
+        h_drain_wait(bar(hDrain), 0);
+      }
+    }
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHHighRegs));
+    // ------------------------------------------------------------ softmax
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t o_addr = tmem + lane_off + kColO;
+    const float sl2 = args.scale_log2;
+    const int w0 = args.w0;
+    float m_used = -INFINITY;
+    float l_sum = 0.f;
+    bool ok = true;
+
+    for (int p = 0; p < npass; ++p) {
+      const int s = p & 1;
+      const uint32_t ph = (uint32_t)(p >> 1) & 1u;
+      ok = mbar_wait(bar(hSFull + s), ph, abort_flag, args.dev_error);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const HPass ps = hilo_pass<kKind>(sc, p);
+      const int mkind = ps.mask;
+      const int dd0 = off - 128 * ps.nb;  // i - j at row 0, column 0
+      const uint32_t s_addr = tmem + lane_off + (uint32_t)(128 * s);
+
+      // S in two 64-column halves: the first half's mask and partial row max
+      // run while the second half's load is in flight.
+      uint32_t sr[4][32];
+      tmem_ld32(s_addr, sr[0]);
+      tmem_ld32(s_addr + 32, sr[1]);
+      tmem_ld_wait(sr[0]);
+      tmem_ld_wait(sr[1]);
+      tmem_ld32(s_addr + 64, sr[2]);
+      tmem_ld32(s_addr + 96, sr[3]);
+
+      float x[128];  // raw scores (fp32 accumulator values)
+      const bool need_mask = mkind == 1 ? (dd0 - 127 < w0)
+                             : mkind == 0 ? (dd0 - 127 < 0 || dd0 + 127 >= w0)
+                                          : (dd0 - 127 < 0);
+      const int dd = dd0 + row;  // i - j = dd - col
+      float m4[4];
+      auto take = [&](int c0) {
+#pragma unroll
+        for (int c = c0; c < c0 + 2; ++c)
+#pragma unroll
+          for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(sr[c][k]);
+        if (need_mask) {
+#pragma unroll
+          for (int col = c0 * 32; col < c0 * 32 + 64; ++col) {
+            const int rel = dd - col;
+            const bool keep = mkind == 1 ? (rel >= w0) : mkind == 0 ? (rel >= 0 && rel < w0) : (rel >= 0);
+            if (!keep) x[col] = -INFINITY;
+          }
+        }
+      };
+      take(0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m4[j] = fmaxf(x[j], x[4 + j]);
+#pragma unroll
+      for (int col = 8; col < 64; col += 8)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m4[j] = fmax3(m4[j], x[col + j], x[col + 4 + j]);
+      // (the partial maxima are tied to this wait, so they are taken while the
+      // second half of S is in flight)
+      asm volatile("tcgen05.wait::ld.sync.aligned;" : "+f"(m4[0]), "+f"(m4[1]), "+f"(m4[2]), "+f"(m4[3])::"memory");
+      tmem_ld_wait(sr[2]);
+      tmem_ld_wait(sr[3]);
+      take(2);
+#pragma unroll
+      for (int col = 64; col < 128; col += 8)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m4[j] = fmax3(m4[j], x[col + j], x[col + 4 + j]);
+      const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+      const float m_new = fmaxf(m_used, mt);
+      float alpha = 1.f;
+      bool rescale_o = false;
+      // Lazy rescaling: keep the exponent offset until the row max has grown
+      // by more than 2^8; p <= 256 stays exact enough in fp32 / bf16.
+      if (m_new > m_used + 8.f) {
+        if (m_used != -INFINITY) {
+          alpha = ex2_approx(m_used - m_new);
+          rescale_o = true;
+        } else {
+          alpha = 0.f;
+        }
+        l_sum *= alpha;
+        m_used = m_new;
+      }
+      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+      // O must be rescaled before this pass's P V; in the (rare) passes that
+      // need it, both halves of P are released after the rescale.
+      const bool resc = __any_sync(0xffffffffu, rescale_o) && p > 0;
+      const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-msub, -msub);
+      uint64_t acc[2] = {0ull, 0ull};
+      auto pair_exp = [&](int half, int k) -> uint32_t {
+        const uint64_t ev = f2_fma(f2_pack(x[half * 64 + 2 * k], x[half * 64 + 2 * k + 1]), sc2, nm2);
+        float e0, e1;
+        f2_unpack(ev, e0, e1);
+        const float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+        acc[k & 1] = f2_add(acc[k & 1], f2_pack(p0, p1));
+        return pack_bf16x2(p0, p1);
+      };
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) pk[k] = pair_exp(0, k);
+        tmem_st32(s_addr, pk);
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pk[k] = pair_exp(1, k);
+        if (!resc) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(hPFull + 2 * s));
+        }
+#pragma unroll
+        for (int k = 8; k < 32; ++k) pk[k] = pair_exp(1, k);
+        tmem_st32(s_addr + 32, pk);
+        if (resc) {
+          // O must hold the previous pass's product first.
+          bool okw = mbar_wait(bar(hPVDone), (uint32_t)(p - 1) & 1u, abort_flag, args.dev_error);
+          okw = __all_sync(0xffffffffu, okw);
+          if (!okw) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(o_addr + c * 32, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+            tmem_st32(o_addr + c * 32, ov);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        if (resc) mbar_arrive(bar(hPFull + 2 * s));
+        mbar_arrive(bar(hPFull + 2 * s + 1));
+      }
+      {
+        float a0, a1;
+        f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+        l_sum += a0 + a1;
+      }
+    }
+
+    if (ok) {
+      ok = mbar_wait(bar(hOFinal), 0, abort_flag, args.dev_error);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int i = mb * 128 + row;  // row of this chunk's Q / O / LSE
+      const float inv = (l_sum > 0.f && npass > 0) ? 1.f / l_sum : 0.f;
+      const size_t obase = (((size_t)b * args.Lq + i) * args.Hq + hq) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(o_addr + c * 32, ov);  // (never written when npass == 0; inv is 0 then)
+        tmem_ld_wait(ov);
+        if (i < args.Lq) {
+          if (args.o_f32 != nullptr) {
+            float4* dst = reinterpret_cast<float4*>(args.o_f32 + obase + c * 32);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float4 w = npass > 0 ? make_float4(__uint_as_float(ov[4 * k]) * inv,
+                                                       __uint_as_float(ov[4 * k + 1]) * inv,
+                                                       __uint_as_float(ov[4 * k + 2]) * inv,
+                                                       __uint_as_float(ov[4 * k + 3]) * inv)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+              dst[k] = w;
+            }
+          } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              w[k] = npass > 0
+                         ? pack_bf16x2(__uint_as_float(ov[2 * k]) * inv, __uint_as_float(ov[2 * k + 1]) * inv)
+                         : 0u;  // no key at all: O = 0, LSE = -inf
+            uint4* dst = reinterpret_cast<uint4*>(args.o + obase + c * 32);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
+        }
+      }
+      if (args.lse != nullptr && i < args.Lq) {
+        const float m = (m_used == -INFINITY) ? 0.f : m_used;
+        args.lse[((size_t)b * args.Hq + hq) * args.Lq + i] =
+            l_sum > 0.f ? (m + __log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHHighRegs));
+    // ------------------------------------------------------------ rotation
+    const int wq = warp & 3;
+    const int e = wq * 32 + lane;  // query row of the block / key row of the tile
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    float2* T1s = reinterpret_cast<float2*>(smem + C::kT1Off);
+    float2* Cs = reinterpret_cast<float2*>(smem + C::kCOff);
+    constexpr int kCElems = H2 * 8;  // float2 per factor buffer
+    const int64_t G = args.G;
+    uint32_t range = 0;
+    bool ok = true;
+
+    // Factor buffer `buf` for a row set whose first row's correction is
+    // `base` (dk_j0 or dq_i0): C[t][a] = R(theta_t (base - 16 a)).  One fp64
+    // sincos per (t, thread); 256 / D threads share a t.
+    auto fill_c = [&](int buf, int64_t base) {
+      constexpr int TPT = 256 / D;
+      constexpr int APT = 8 / TPT;
+      const int t = e / TPT;
+      const int a0 = (e % TPT) * APT;
+      double sn, cs;
+      sincos(args.theta[t] * (double)base, &sn, &cs);
+      const float cb = (float)cs, sb = (float)sn;
+#pragma unroll
+      for (int j = 0; j < APT; ++j) {
+        const float2 m = args.t16[t * 8 + a0 + j];
+        Cs[buf * kCElems + ((t >> 1) * 8 + a0 + j) * 2 + (t & 1)] = make_float2(cb * m.x - sb * m.y, cb * m.y + sb * m.x);
+      }
+    };
+    // Position offset of row e of a row set starting at position x0 from the
+    // set's first row: f(x0 + e) - f(x0) - e = -delta, delta in [0, 127].
+    auto delta_of = [&](int64_t x0) -> int { return e - (int)((x0 % G + e) / G); };
+
+    uint32_t raw[H2];  // one row of bf16 pairs
+    auto load_row = [&](const __nv_bfloat16* src, bool valid) {
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+      for (int w = 0; w < H2 / 4; ++w) {
+        const uint4 v = valid ? __ldg(s4 + w) : make_uint4(0u, 0u, 0u, 0u);
+        raw[4 * w] = v.x;
+        raw[4 * w + 1] = v.y;
+        raw[4 * w + 2] = v.z;
+        raw[4 * w + 3] = v.w;
+      }
+    };
+    const int qi = mb * 128 + e;  // this thread's query row in the chunk
+    const __nv_bfloat16* qrow = args.q + (((size_t)b * args.Lq + qi) * args.Hq + hq) * D;
+    // The query operands of the base (local) passes: the base row, as bf16.
+    auto write_base_q = [&]() {
+#pragma unroll
+      for (int U = 0; U < D / 8; ++U)
+        tmem_st4(tmem + lane_off + kColQA + 4 * U, raw[4 * U], raw[4 * U + 1], raw[4 * U + 2], raw[4 * U + 3]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(hQReady));
+    };
+
+    // Tables (R(-theta_t b) from the arguments) and the query block's factors.
+    for (int i = e; i < H2 * 16; i += 128) {
+      const int t = i >> 4, bb = i & 15;
+      T1s[((t >> 1) * 16 + bb) * 2 + (t & 1)] = args.t1[i];
+    }
+    const int64_t dq0 = off / G + args.shift - off;  // dq at the block's first query
+    fill_c(2, dq0);
+    mbar_arrive(bar(hCReady));
+    ok = mbar_wait(bar(hCReady), 0, abort_flag, args.dev_error);
+    int c_phase = 1;
+
+    // Query operands of the first pass kind.
+    if (ok && npass > 0) {
+      load_row(qrow, qi < args.Lq);
+      if (hilo_pass<kKind>(sc, 0).remote) {
+        rotate_row_hilo<D>(raw, Cs + 2 * kCElems, T1s, delta_of(off), range,
+                           [&](int U, const uint32_t (&h)[4], const uint32_t (&l)[4]) {
+                             tmem_st4(tmem + lane_off + kColQA + 4 * U, h[0], h[1], h[2], h[3]);
+                             tmem_st4(tmem + lane_off + kColQB + 4 * U, l[0], l[1], l[2], l[3]);
+                           });
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(hQReady));
+      } else {
+        write_base_q();
+      }
+    }
+
+    if (kRotK) {
+      // Key tiles, one ahead: the next tile's rows are loaded (and its factors
+      // formed) while the tensor core still reads the stage they will fill.
+      auto key_row = [&](int nb) -> const __nv_bfloat16* {
+        const int j = nb * 128 + e;
+        return args.k + (((size_t)b * args.k_rows + (j < args.k_rows ? j : 0)) * args.Hkv + kvh) * D;
+      };
+      auto prep = [&](int p) -> bool {
+        const HPass ps = hilo_pass<kKind>(sc, p);
+        load_row(key_row(ps.nb), ps.nb * 128 + e < args.k_rows);
+        if (ps.remote) {
+          const int64_t j0 = (int64_t)ps.nb * 128;
+          fill_c(p & 1, j0 / G - j0);
+        }
+        mbar_arrive(bar(hCReady));
+        const bool w = mbar_wait(bar(hCReady), (uint32_t)c_phase & 1u, abort_flag, args.dev_error);
+        ++c_phase;
+        return w;
+      };
+      if (ok && npass > 0) ok = prep(0);
+      for (int p = 0; p < npass && ok; ++p) {
+        const int s = p & 1;
+        const HPass ps = hilo_pass<kKind>(sc, p);
+        if (!(ok = mbar_wait(bar(hKEmpty + s), ((uint32_t)(p >> 1) & 1u) ^ 1u, abort_flag, args.dev_error))) break;
+        const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
+        const uint32_t rowoff = (uint32_t)(e * 128);
+        const uint32_t sw = (uint32_t)(e & 7);
+        auto unit_addr = [&](uint32_t slot, int U) -> uint32_t {
+          return slot + (uint32_t)((U >> 3) * kSlab) + rowoff + ((((uint32_t)U & 7u) ^ sw) << 4);
+        };
+        if (ps.remote) {
+          const int64_t j0 = (int64_t)ps.nb * 128;
+          rotate_row_hilo<D>(raw, Cs + (p & 1) * kCElems, T1s, delta_of(j0), range,
+                             [&](int U, const uint32_t (&h)[4], const uint32_t (&l)[4]) {
+                               sts128(unit_addr(khi, U), h[0], h[1], h[2], h[3]);
+                               sts128(unit_addr(khi + C::kTile, U), l[0], l[1], l[2], l[3]);
+                             });
+        } else {
+#pragma unroll
+          for (int U = 0; U < D / 8; ++U)
+            sts128(unit_addr(khi, U), raw[4 * U], raw[4 * U + 1], raw[4 * U + 2], raw[4 * U + 3]);
+        }
+        fence_proxy_async_smem();  // the tensor core reads these rows through the async proxy
+        mbar_arrive(bar(hKFull + s));
+        if (q_switch && p == p_switch) {
+          // The remote query operands have been read for the last time: put
+          // the base rows in their place.
+          if (!(ok = mbar_wait(bar(hQEmpty), 0, abort_flag, args.dev_error))) break;
+          tc_fence_after();
+          load_row(qrow, qi < args.Lq);
+          write_base_q();
+        }
+        if (p + 1 < npass && !(ok = prep(p + 1))) break;
+      }
+    } else if (ok && q_switch) {
+      ok = mbar_wait(bar(hQEmpty), 0, abort_flag, args.dev_error);
+      if (ok) {
+        tc_fence_after();
+        load_row(qrow, qi < args.Lq);
+        write_base_q();
+      }
+    }
+    // A corrected value beyond fp16's range (|x| >= 65520) makes the result
+    // invalid; report it.
+    if ((range & 0x80008000u) != 0u && args.dev_error != nullptr) atomicExch(args.dev_error, kDevRange);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512u);
+}
+
+template <int D, bool kRotK, int kKind>
+cudaError_t launch_hilo_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_kh,
+                          const CUtensorMap& tm_kl, const PrefillHiloArgs& a, cudaStream_t stream) {
+  auto k = bifocal_prefill_hilo_kernel<D, kRotK, kKind>;
+  // The setmaxnreg split inside the kernel assumes the launch register count.
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, k);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs != kHLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, HCfg<D>::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.Hq, a.num_mb, a.B);
+  k<<<grid, kHThreads, HCfg<D>::kSmem, stream>>>(tm_k, tm_v, tm_kh, tm_kl, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_hilo_d(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_kh,
+                          const CUtensorMap& tm_kl, const PrefillHiloArgs& a, bool rot_k, cudaStream_t stream) {
+  if (!rot_k) {
+    if (a.kind != kBifocal) return cudaErrorInvalidValue;
+    return launch_hilo_t<D, false, kBifocal>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+  }
+  switch (a.kind) {
+    case kWindowBase: return launch_hilo_t<D, true, kWindowBase>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    case kCausalRemote: return launch_hilo_t<D, true, kCausalRemote>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    case kWindowRemote: return launch_hilo_t<D, true, kWindowRemote>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    default: return launch_hilo_t<D, true, kBifocal>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_hilo(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_kh,
+                                const CUtensorMap& tm_kl, const PrefillHiloArgs& a, int D, bool rot_k,
+                                cudaStream_t stream) {
+  return D == 128 ? launch_hilo_d<128>(tm_k, tm_v, tm_kh, tm_kl, a, rot_k, stream)
+                  : launch_hilo_d<64>(tm_k, tm_v, tm_kh, tm_kl, a, rot_k, stream);
+}
+
+}  // namespace jl

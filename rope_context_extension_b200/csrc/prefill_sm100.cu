@@ -6,6 +6,11 @@
 // "Method"; gist.science summary, "Methodologie §1").  The remote rows come
 // from the correction pass in rope_rotate.cu, in fp16; local products are
 // bf16 x bf16, remote ones fp16 x fp16, P V is bf16 x bf16, all fp32-accumulated.
+// This is the fast, lower-precision path (one fp16 product per remote score,
+// about 2^-11 relative operand error); prefill_hilo_sm100.cu is the default.
+// With every pair local (G = 1 or w0 >= L) it is plain causal RoPE attention
+// on the bf16 inputs, exact up to accumulation order, and serves that case for
+// every precision.
 //
 // Instead of the pages' three FlashAttention calls merged by inclusion-exclusion,
 // each 128x128 (query block, key block) tile is classified by its range of
@@ -23,10 +28,6 @@
 //   warps 8-11  softmax for head 1
 // TMEM columns: S_h at 128 h, O_h at 128 NH + D h.  P (bf16) overwrites the
 // first 64 columns of S_h and is the A operand of O_h += P V from TMEM.
-// Split mode (opt-in, for inputs with large-norm keys): the corrected rows
-// come as fp16 hi + lo pairs and a remote S accumulates Q_hi K_hi + Q_hi K_lo
-// + Q_lo K_hi (about 2^-21 relative error instead of 2^-12), one query head per
-// CTA so that Q_hi / Q_lo and K_hi / K_lo fit in shared memory.
 // Per pass the MMA order is S0(i), PV1(i-1), S1(i), PV0(i): each softmax group
 // works on its S while the tensor core runs the other head's two products.
 #include "jl_kernels.cuh"
@@ -45,15 +46,12 @@ constexpr int kHighRegs = 200;    // warpgroups 1-2: softmax
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kChunkBytes = 128 * 128;  // one 128-row x 128-byte swizzled slab
 
-// kSplit: remote scores from fp16 hi + lo corrected rows (one query head per
-// CTA; the Q region holds Q_hi and Q_lo, each K stage K_hi and K_lo, and V is
-// single-buffered to fit shared memory).
-template <int D, bool kSplit>
+template <int D>
 struct Cfg {
   static constexpr int kChunks = D / 64;  // 64-element (128 B) slabs per row
   static constexpr int kTileBytes = kBM * D * 2;
-  static constexpr int kKSlots = kSplit ? 2 : 1;   // tiles per K stage
-  static constexpr int kVStages = kSplit ? 1 : kStages;
+  static constexpr int kKSlots = 1;   // tiles per K stage
+  static constexpr int kVStages = kStages;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kKSlots * kTileBytes;
@@ -90,13 +88,13 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-template <int D, bool kSplit, int kKind>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
-                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qr_lo,
-                           const __grid_constant__ CUtensorMap tm_kr_lo, const PrefillArgs args) {
-  using C = Cfg<D, kSplit>;
+                           const __grid_constant__ CUtensorMap tm_v, const PrefillArgs args) {
+  constexpr int kKind = kBifocal;
+  using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -175,22 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_kr);
       tma_prefetch_map(&tm_v);
-      if (kSplit) {
-        tma_prefetch_map(&tm_qr_lo);
-        tma_prefetch_map(&tm_kr_lo);
-      }
-      // Q region: one tile per head (NH heads), or Q_hi / Q_lo of the single
-      // head for remote passes in split mode.
+      // Q region: one tile per head (NH heads).
       auto load_q = [&](bool remote) {
-        if (kSplit && remote) {
-          mbar_arrive_expect_tx(bar(kQFull), (uint32_t)(2 * C::kTileBytes));
-          for (int c = 0; c < C::kChunks; ++c) {
-            tma_load_4d(sbase + C::kQOff + c * kChunkBytes, &tm_qr, bar(kQFull), c * 64, hq0, mb * kBM, b);
-            tma_load_4d(sbase + C::kQOff + C::kTileBytes + c * kChunkBytes, &tm_qr_lo, bar(kQFull), c * 64, hq0,
-                        mb * kBM, b);
-          }
-          return;
-        }
         const CUtensorMap* m = remote ? &tm_qr : &tm_q;
         mbar_arrive_expect_tx(bar(kQFull), (uint32_t)(NH * C::kTileBytes));
         for (int hh = 0; hh < NH; ++hh)
@@ -217,14 +201,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!(ok = mbar_wait(bar(kKEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
         const uint32_t kdst = sbase + C::kKOff + s * C::kKSlots * C::kTileBytes;
-        const bool two = kSplit && remote;
-        mbar_arrive_expect_tx(bar(kKFull + s), (uint32_t)((two ? 2 : 1) * C::kTileBytes));
-        for (int c = 0; c < C::kChunks; ++c) {
+        mbar_arrive_expect_tx(bar(kKFull + s), (uint32_t)C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
           tma_load_4d(kdst + c * kChunkBytes, remote ? &tm_kr : &tm_k, bar(kKFull + s), c * 64, kvh, nb * kBN, b);
-          if (two)
-            tma_load_4d(kdst + C::kTileBytes + c * kChunkBytes, &tm_kr_lo, bar(kKFull + s), c * 64, kvh, nb * kBN,
-                        b);
-        }
         k_last = p;
         if (!(ok = mbar_wait(bar(kVEmpty + sv), phv ^ 1u, abort_flag, args.dev_error))) break;
         mbar_arrive_expect_tx(bar(kVFull + sv), (uint32_t)C::kTileBytes);
@@ -269,21 +248,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
           mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
                  id_s, ks > 0 ? 1u : 0u);
-        }
-        if (kSplit && remote) {
-          // + Q_hi K_lo + Q_lo K_hi into the same accumulator
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
-            mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + off, 16, 1024),
-                   make_sdesc_sw128(ka + C::kTileBytes + off, 16, 1024), id_s, 1u);
-          }
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
-            mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + C::kTileBytes + off, 16, 1024),
-                   make_sdesc_sw128(ka + off, 16, 1024), id_s, 1u);
-          }
         }
         tc_commit(bar(kSFull + h));
         if (h == NH - 1) {
@@ -536,52 +500,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
-template <int D, bool kSplit, int kKind>
+template <int D>
 cudaError_t launch_prefill_t(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
-                             const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
-                             const CUtensorMap& tm_kr_lo, const PrefillArgs& a, cudaStream_t stream) {
-  auto k = bifocal_prefill_kernel<D, kSplit, kKind>;
+                             const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const PrefillArgs& a,
+                             cudaStream_t stream) {
+  auto k = bifocal_prefill_kernel<D>;
   // The setmaxnreg split inside the kernel assumes the launch register count.
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, k);
   if (e != cudaSuccess) return e;
   if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, kSplit>::kSmem);
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Hq / a.nh, a.num_mb, a.B);
-  k<<<grid, kThreads, Cfg<D, kSplit>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a);
+  k<<<grid, kThreads, Cfg<D>::kSmem, stream>>>(tm_q, tm_qr, tm_k, tm_kr, tm_v, a);
   return cudaGetLastError();
-}
-
-template <int D, bool kSplit>
-cudaError_t launch_prefill_kind(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
-                                const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
-                                const CUtensorMap& tm_kr_lo, const PrefillArgs& a, cudaStream_t stream) {
-  switch (a.kind) {
-    case kWindowBase:
-      return launch_prefill_t<D, kSplit, kWindowBase>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
-    case kCausalRemote:
-      return launch_prefill_t<D, kSplit, kCausalRemote>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a,
-                                                        stream);
-    case kWindowRemote:
-      return launch_prefill_t<D, kSplit, kWindowRemote>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a,
-                                                        stream);
-    default:
-      return launch_prefill_t<D, kSplit, kBifocal>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
-  }
 }
 
 }  // namespace
 
 cudaError_t launch_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_qr, const CUtensorMap& tm_k,
-                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const CUtensorMap& tm_qr_lo,
-                           const CUtensorMap& tm_kr_lo, const PrefillArgs& a, int D, bool split,
+                           const CUtensorMap& tm_kr, const CUtensorMap& tm_v, const PrefillArgs& a, int D,
                            cudaStream_t stream) {
-  if (D == 128)
-    return split ? launch_prefill_kind<128, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
-                 : launch_prefill_kind<128, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
-  return split ? launch_prefill_kind<64, true>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream)
-               : launch_prefill_kind<64, false>(tm_q, tm_qr, tm_k, tm_kr, tm_v, tm_qr_lo, tm_kr_lo, a, stream);
+  return D == 128 ? launch_prefill_t<128>(tm_q, tm_qr, tm_k, tm_kr, tm_v, a, stream)
+                  : launch_prefill_t<64>(tm_q, tm_qr, tm_k, tm_kr, tm_v, a, stream);
 }
 
 }  // namespace jl

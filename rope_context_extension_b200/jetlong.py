@@ -14,7 +14,7 @@ import os
 import numpy as np
 
 __all__ = [
-    "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JL_REMOTE_SPLIT", "JetLongError", "lib", "library_path",
+    "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JL_PREFILL_FP16", "JL_PREFILL_PREROTATED_K", "JetLongError", "lib", "library_path",
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
@@ -25,7 +25,11 @@ __all__ = [
 
 JL_QSHIFT_NONE = 0
 JL_QSHIFT_SELF_EXTEND = 1
-JL_REMOTE_SPLIT = 2  # OR into mode: fp16 hi + lo remote operands in prefill (twice the workspace)
+# Optional prefill flags OR-ed into mode (include/jl_api.h): the default corrects Q
+# and K inside the attention kernel with fp16 hi + lo remote operands and needs no
+# workspace.
+JL_PREFILL_FP16 = 4          # one fp16 product per remote score from pre-rotated rows (needs workspace)
+JL_PREFILL_PREROTATED_K = 8  # default arithmetic, key rows' hi / lo from a correction pass (needs workspace)
 EXPORTED_SYMBOLS = (
     "jl_status_string", "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes",
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
@@ -73,8 +77,8 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_prefill.restype = c_i
     L.jl_prefill_correction.argtypes = [c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_i, c_p, c_sz, c_p]
     L.jl_prefill_correction.restype = c_i
-    L.jl_prefill_attention.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_f, c_i, c_p,
-                                       c_sz, c_p, c_p]
+    L.jl_prefill_attention.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_f, c_i,
+                                       c_p, c_sz, c_p, c_p]
     L.jl_prefill_attention.restype = c_i
     L.jl_bifocal_decode.argtypes = [c_p, c_p, c_p, c_i64, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_f,
                                     c_i, c_p, c_sz, c_p, c_p]
@@ -170,8 +174,9 @@ def jl_bifocal_prefill(q, k, v, o, lse, *, w0: int, w_pretrained: int, rope_base
                        softmax_scale: float = 0.0, mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None,
                        dev_error=None, stream=None):
     """Fused bifocal prefill.  q [B, L, Hq, D], k / v [B, L, Hkv, D], o like q (bf16, CUDA);
-    lse [B, Hq, L] fp32 or None; workspace: uint8 CUDA tensor of
-    jl_prefill_workspace_bytes(...) bytes (may be None when every pair is local)."""
+    lse [B, Hq, L] fp32 or None; workspace: None in the default mode, else a uint8 CUDA
+    tensor of jl_prefill_workspace_bytes(...) bytes (JL_PREFILL_FP16 /
+    JL_PREFILL_PREROTATED_K)."""
     import torch
     B, L, Hq, D = q.shape
     Hkv = k.shape[2]
@@ -202,8 +207,9 @@ def jl_prefill_correction(q, k, *, w0: int, w_pretrained: int, rope_base: float,
     _check(st, "jl_prefill_correction")
 
 
-def jl_prefill_attention(q, k, v, o, lse, *, w0: int, w_pretrained: int, softmax_scale: float = 0.0,
-                         mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None, dev_error=None, stream=None):
+def jl_prefill_attention(q, k, v, o, lse, *, w0: int, w_pretrained: int, rope_base: float,
+                         softmax_scale: float = 0.0, mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None,
+                         dev_error=None, stream=None):
     """Stage 2 of jl_bifocal_prefill: the fused attention kernel."""
     import torch
     B, L, Hq, D = q.shape
@@ -216,8 +222,8 @@ def jl_prefill_attention(q, k, v, o, lse, *, w0: int, w_pretrained: int, softmax
         _check_tensor(lse, "lse", torch.float32, (B, Hq, L))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().jl_prefill_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, L, Hq, Hkv, D, int(w0),
-                                    int(w_pretrained), float(softmax_scale), int(mode), _ptr(workspace), ws_bytes,
-                                    _ptr(dev_error), _stream(stream))
+                                    int(w_pretrained), float(rope_base), float(softmax_scale), int(mode),
+                                    _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream))
     _check(st, "jl_prefill_attention")
 
 

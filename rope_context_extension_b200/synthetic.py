@@ -21,11 +21,23 @@ from __future__ import annotations
 
 import torch
 
-__all__ = ["prefill_inputs", "decode_inputs", "scale_key_outliers"]
+__all__ = ["prefill_inputs", "decode_inputs", "scale_key_outliers", "outlier_rows"]
 
 
 def _randn_bf16(gen: torch.Generator, shape) -> torch.Tensor:
     return torch.randn(*shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+
+
+def outlier_rows(B: int, n: int, Hkv: int, frac: float, seed: int = 1):
+    """The seeded (b, j, kv_head) index triples ``scale_key_outliers`` picks among
+    the first ``n`` keys of a [B, *, Hkv, d] key tensor (three int64 tensors)."""
+    total = B * n * Hkv
+    count = max(1, int(round(frac * total)))
+    gen = torch.Generator("cpu").manual_seed(seed)
+    idx = torch.randperm(total, generator=gen)[:count]
+    b = idx // (n * Hkv)
+    rem = idx % (n * Hkv)
+    return b, rem // Hkv, rem % Hkv
 
 
 def scale_key_outliers(k: torch.Tensor, frac: float, scale: float = 8.0, seed: int = 1,
@@ -38,15 +50,7 @@ def scale_key_outliers(k: torch.Tensor, frac: float, scale: float = 8.0, seed: i
     if frac <= 0.0:
         return k
     B, Lmax, Hkv, _ = k.shape
-    n = Lmax if length is None else length
-    total = B * n * Hkv
-    count = max(1, int(round(frac * total)))
-    gen = torch.Generator("cpu").manual_seed(seed)
-    idx = torch.randperm(total, generator=gen)[:count]
-    b = idx // (n * Hkv)
-    rem = idx % (n * Hkv)
-    j = rem // Hkv
-    h = rem % Hkv
+    b, j, h = outlier_rows(B, Lmax if length is None else length, Hkv, frac, seed)
     k[b, j, h, :] = (k[b, j, h, :].float() * scale).to(torch.bfloat16)
     return k
 

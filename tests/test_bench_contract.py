@@ -44,7 +44,7 @@ def test_reference_arm_json_line():
 @pytest.mark.gpu
 def test_our_arm_json_line_small():
     d = _run(["--steps", "3", "--warmup", "3", "--prefill-len", "8192", "--decode-len", "8192", "--cpu-seconds", "2",
-              "--no-split", "--no-ie"], timeout=900)
+              "--no-variants", "--no-ie", "--no-other-workloads"], timeout=900)
     assert BASE_KEYS <= set(d)
     assert d["n_gpus"] == 1 and d["steps"] == 3 and d["warmup"] == 3 and d["scaling"] == "weak"
     assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["dtype"] == "bf16"

@@ -14,7 +14,7 @@ import torch
 from oracle import jetlong_oracle as jo
 from rope_context_extension_b200 import jetlong as jl
 from rope_context_extension_b200 import synthetic
-from tests.gpu_helpers import MODES, assert_close
+from tests.gpu_helpers import PRECISIONS, prefill_workspace, MODES, assert_close
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
@@ -26,15 +26,14 @@ def _built():
     build.build()
 
 
-def _chunk(q, kc, vc, P, w0, W, base, mode=jo.MODE_SELF_EXTEND, split=False):
+def _chunk(q, kc, vc, P, w0, W, base, mode=jo.MODE_SELF_EXTEND, prec="default"):
     B, C, Hq, D = q.shape
     Hkv = kc.shape[2]
     o = torch.empty_like(q)
     lse = torch.empty(B, Hq, C, dtype=torch.float32, device=DEV)
-    ws = torch.empty(jl.jl_prefill_chunk_workspace_bytes(B, P, C, Hq, Hkv, D) * (2 if split else 1),
-                     dtype=torch.uint8, device=DEV)
+    ws = prefill_workspace(prec, jl.jl_prefill_chunk_workspace_bytes(B, P, C, Hq, Hkv, D), DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
-    m = MODES[mode] | (jl.JL_REMOTE_SPLIT if split else 0)
+    m = MODES[mode] | PRECISIONS[prec]
     jl.jl_bifocal_prefill_chunk(q, kc, vc, o, lse, q_offset=P, w0=w0, w_pretrained=W, rope_base=base, mode=m,
                                 workspace=ws, dev_error=err)
     torch.cuda.synchronize()
@@ -55,20 +54,21 @@ def _oracle_chunk(q_full, k, v, P, C, w0, W, base, mode=jo.MODE_SELF_EXTEND):
     return o, lse
 
 
-@pytest.mark.parametrize("P,C,w0,W,mode,split", [
-    (0, 1500, 200, 400, jo.MODE_SELF_EXTEND, False),     # whole sequence from a cache
-    (700, 800, 200, 400, jo.MODE_SELF_EXTEND, False),    # offset not a multiple of the 128-row tile
-    (1300, 200, 200, 400, jo.MODE_NONE, False),
-    (1111, 389, 0, 400, jo.MODE_SELF_EXTEND, False),     # w0 = 0: every pair remote
-    (5, 50, 16, 20, jo.MODE_SELF_EXTEND, False),         # small chunk, stale rows after it in the cache
-    (900, 600, 200, 1600, jo.MODE_SELF_EXTEND, False),   # G = 1 at the total length: plain causal RoPE
-    (700, 800, 200, 400, jo.MODE_SELF_EXTEND, True),     # split-precision remote scores
+@pytest.mark.parametrize("P,C,w0,W,mode,prec,outl", [
+    (0, 1500, 200, 400, jo.MODE_SELF_EXTEND, "default", 0.01),   # whole sequence from a cache
+    (700, 800, 200, 400, jo.MODE_SELF_EXTEND, "default", 0.01),  # offset not a multiple of the 128-row tile
+    (1300, 200, 200, 400, jo.MODE_NONE, "default", 0.0),
+    (1111, 389, 0, 400, jo.MODE_SELF_EXTEND, "default", 0.01),   # w0 = 0: every pair remote
+    (5, 50, 16, 20, jo.MODE_SELF_EXTEND, "default", 0.0),        # small chunk, stale rows after it in the cache
+    (900, 600, 200, 1600, jo.MODE_SELF_EXTEND, "default", 0.0),  # G = 1 at the total length: plain causal RoPE
+    (700, 800, 200, 400, jo.MODE_SELF_EXTEND, "prerot", 0.01),   # key rows' hi / lo from the correction pass
+    (700, 800, 200, 400, jo.MODE_SELF_EXTEND, "fp16", 0.0),      # single fp16 product
 ])
-def test_chunk_matches_oracle(P, C, w0, W, mode, split):
+def test_chunk_matches_oracle(P, C, w0, W, mode, prec, outl):
     Lmax = P + C + 77
-    q_full, k, v = synthetic.prefill_inputs(1, Lmax, 8, 2, 128, seed=P + C, outlier_frac=0.0)
+    q_full, k, v = synthetic.prefill_inputs(1, Lmax, 8, 2, 128, seed=P + C, outlier_frac=outl)
     qc = q_full[:, P:P + C].contiguous()
-    o, lse = _chunk(qc.to(DEV), k.to(DEV), v.to(DEV), P, w0, W, 1e6, mode, split)
+    o, lse = _chunk(qc.to(DEV), k.to(DEV), v.to(DEV), P, w0, W, 1e6, mode, prec)
     o_ref, lse_ref = _oracle_chunk(q_full, k, v, P, C, w0, W, 1e6, mode)
     assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"chunk P{P} C{C}")
 
@@ -81,8 +81,7 @@ def test_final_chunk_equals_whole_prefill_rows():
     qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
     o_full = torch.empty_like(qd)
     lse_full = torch.empty(1, 8, L, dtype=torch.float32, device=DEV)
-    ws = torch.empty(jl.jl_prefill_workspace_bytes(1, L, 8, 2, 128), dtype=torch.uint8, device=DEV)
-    jl.jl_bifocal_prefill(qd, kd, vd, o_full, lse_full, w0=w0, w_pretrained=W, rope_base=1e6, workspace=ws)
+    jl.jl_bifocal_prefill(qd, kd, vd, o_full, lse_full, w0=w0, w_pretrained=W, rope_base=1e6)
     kbig = torch.cat([kd, torch.full((1, 300, 2, 128), 7.0, dtype=torch.bfloat16, device=DEV)], dim=1)
     vbig = torch.cat([vd, torch.full((1, 300, 2, 128), -7.0, dtype=torch.bfloat16, device=DEV)], dim=1)
     o_c, lse_c = _chunk(qd[:, P:].contiguous(), kbig, vbig, P, w0, W, 1e6)

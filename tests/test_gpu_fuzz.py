@@ -14,7 +14,7 @@ import torch
 from oracle import jetlong_oracle as jo
 from rope_context_extension_b200 import jetlong as jl
 from rope_context_extension_b200 import synthetic
-from tests.gpu_helpers import LSE_MAX_ABS, MODES, assert_close, run_decode, run_prefill
+from tests.gpu_helpers import MODES, assert_close, run_decode, run_prefill
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
@@ -45,8 +45,10 @@ def _prefill_cases(n=40, seed=2024):
         L = int(rng.integers(1, 641))
         D, Hq, Hkv, W, w0, mode = _draw(rng, L)
         B = int(rng.integers(1, 3))
-        split = bool(rng.random() < 0.3)
-        cases.append((B, L, Hq, Hkv, D, W, w0, mode, split))
+        u = rng.random()
+        prec = "prerot" if u < 0.2 else ("fp16" if u < 0.35 else "default")
+        outl = 0.0 if prec == "fp16" else float(rng.choice([0.0, 0.01]))
+        cases.append((B, L, Hq, Hkv, D, W, w0, mode, prec, outl))
     return cases
 
 
@@ -62,15 +64,15 @@ def _decode_cases(n=40, seed=7):
     return cases
 
 
-@pytest.mark.parametrize("B,L,Hq,Hkv,D,W,w0,mode,split", _prefill_cases())
-def test_prefill_random_shapes(B, L, Hq, Hkv, D, W, w0, mode, split):
-    q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=L * 7 + Hq)
-    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=10000.0, mode=mode, split=split)
+@pytest.mark.parametrize("B,L,Hq,Hkv,D,W,w0,mode,prec,outl", _prefill_cases())
+def test_prefill_random_shapes(B, L, Hq, Hkv, D, W, w0, mode, prec, outl):
+    q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=L * 7 + Hq, outlier_frac=outl)
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=10000.0, mode=mode, prec=prec)
     assert err == 0
     p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=10000.0, mode=mode)
     o_ref, lse_ref = jo.prefill_dense(q.float().numpy(), k.float().numpy(), v.float().numpy(), p)
-    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"B{B} L{L} {Hq}/{Hkv} d{D} W{W} w0{w0} {mode} split{split}",
-                 lse_tol=LSE_MAX_ABS)
+    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref,
+                 f"B{B} L{L} {Hq}/{Hkv} d{D} W{W} w0{w0} {mode} {prec} outliers {outl}")
 
 
 @pytest.mark.parametrize("B,Lmax,L,Hq,Hkv,D,W,w0,mode", _decode_cases())
@@ -102,10 +104,9 @@ def test_chunked_prefill_random_shapes(P, C, Hq, Hkv, D, W, w0, mode):
     kd, vd = k.to(DEV), v.to(DEV)
     o = torch.empty_like(q)
     lse = torch.empty(1, Hq, C, dtype=torch.float32, device=DEV)
-    ws = torch.empty(jl.jl_prefill_chunk_workspace_bytes(1, P, C, Hq, Hkv, D), dtype=torch.uint8, device=DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
     jl.jl_bifocal_prefill_chunk(q, kd, vd, o, lse, q_offset=P, w0=w0, w_pretrained=W, rope_base=10000.0,
-                                mode=MODES[mode], workspace=ws, dev_error=err)
+                                mode=MODES[mode], dev_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     p = jo.BifocalParams(L=P + C, w0=w0, w_pretrained=W, base=10000.0, mode=mode)
