@@ -3,16 +3,18 @@
 One step = one pass of the whole hot path over one batch of synthetic input:
   * prefill of the Qwen3-8B-shaped layer at 128K (batch 1, 32 q heads / 8 kv
     heads, head_dim 128, RoPE base 1e6, L 131072, w_pretrained 32768 -> G 4,
-    w0 4096) through the default path: one fused tcgen05 kernel that applies
-    the correction rotations itself and carries remote scores as fp16 hi + lo
-    products (the path held to the oracle's tolerances on every workload);
+    w0 4096) through the default path (the one held to the oracle's
+    tolerances on every workload): the key-row correction pass, then the fused
+    tcgen05 kernel that corrects the query block itself and carries remote
+    scores as fp16 hi + lo products;
   * decode of the Qwen3-4B-shaped layer at 128K (32 / 8 heads, head_dim 128,
     batch 8, cache of 131072 base-rotated keys, G 4, w0 4096).
 `value` is the prefill TFLOP/s (algorithmic 4 * B * Hq * d * L(L+1)/2 per
 step, summed over ranks, divided by the max-over-ranks device time of the
 prefill calls); the decode GB/s (K and V bytes read once) is reported beside
-it, and so are the other prefill paths (single fp16 product, pre-rotated key
-rows, the three-call inclusion-exclusion formulation, plain RoPE), the
+it, and so are the other prefill paths (single fp16 product, key tiles
+corrected inside the kernel, the three-call inclusion-exclusion formulation,
+plain RoPE), the
 Qwen3-1.7B 64K and tiny workloads and the length / band sweep.  Inputs are
 larger than L2 (1 GiB Q, 4 GiB KV cache), so no flush runs between steps.
 
@@ -268,6 +270,8 @@ def run_ours(args):
     o = torch.empty_like(q)
     lse = torch.empty(P["B"], P["Hq"], P["L"], dtype=torch.float32, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(jl.jl_prefill_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]), dtype=torch.uint8,
+                     device=dev)
     # decode buffers
     dq = gen_on_device((Dc["B"], Dc["Hq"], Dc["D"]), seed + 3, dev)
     kc = gen_on_device((Dc["B"], Dc["L"], Dc["Hkv"], Dc["D"]), seed + 4, dev)
@@ -277,13 +281,14 @@ def run_ours(args):
     dws = torch.zeros(jl.jl_decode_workspace_bytes(Dc["B"], Dc["L"], Dc["Hq"], Dc["Hkv"], Dc["D"]),
                       dtype=torch.uint8, device=dev)
 
-    def prefill_step(evs=None, w0=None, mode=SE, wsp=None):
-        # stage 1 (the correction pass) launches nothing in the default mode
+    def prefill_step(evs=None, w0=None, mode=SE, wsp=ws):
+        # stage 1: the correction pass (the key rows' hi / lo parts); stage 2:
+        # the attention kernel
         w = P["w0"] if w0 is None else w0
         if evs:
             evs[0].record(stream)
         jl.jl_prefill_correction(q, k, w0=w, w_pretrained=P["W"], rope_base=P["base"], mode=mode, workspace=wsp,
-                                 stream=stream)
+                                 dev_error=err, stream=stream)
         if evs:
             evs[1].record(stream)
         jl.jl_prefill_attention(q, k, v, o, lse, w0=w, w_pretrained=P["W"], rope_base=P["base"], mode=mode,
@@ -400,22 +405,19 @@ def run_ours(args):
     plain_pre_ms = time_calls(lambda: prefill_step(w0=P["L"]), max(2, K // 2))
     plain_dec_ms = time_calls(lambda: decode_step(w0=Dc["L"]), max(2, K // 2))
     # the other prefill paths on the same inputs
-    ws_opt = torch.empty(jl.jl_prefill_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]), dtype=torch.uint8,
-                         device=dev)
     paths = {}
     for name, flag in (("fp16_single_product", jl.JL_PREFILL_FP16),
-                       ("prerotated_keys", jl.JL_PREFILL_PREROTATED_K)):
+                       ("keys_corrected_in_kernel", jl.JL_PREFILL_KEYS_IN_KERNEL)):
         if args.no_variants:
             break
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        ms = time_calls(lambda: prefill_step(mode=SE | flag, wsp=ws_opt), 2)
-        prefill_step(evs, mode=SE | flag, wsp=ws_opt)
+        ms = time_calls(lambda: prefill_step(mode=SE | flag), 2)
+        prefill_step(evs, mode=SE | flag)
         torch.cuda.synchronize()
         paths[name] = {"ms": round(ms, 3), "tflops": round(flop / (ms * 1e-3) / 1e12, 2),
                        "correction_ms": round(evs[0].elapsed_time(evs[1]), 3),
                        "attention_ms": round(evs[1].elapsed_time(evs[2]), 3),
                        "speed_vs_default": round(pre_ms_max / ms, 3)}
-    del ws_opt
     ie = None
     if not args.no_ie:
         ws3 = torch.empty(jl.jl_prefill_ie_workspace_bytes(P["B"], P["L"], P["Hq"], P["Hkv"], P["D"]),
@@ -440,18 +442,20 @@ def run_ours(args):
             v2 = gen_on_device((c["B"], c["L"], c["Hkv"], c["D"]), seed + 13, dev)
             o2 = torch.empty_like(q2)
             l2 = torch.empty(c["B"], c["Hq"], c["L"], dtype=torch.float32, device=dev)
+            w2 = torch.empty(jl.jl_prefill_workspace_bytes(c["B"], c["L"], c["Hq"], c["Hkv"], c["D"]),
+                             dtype=torch.uint8, device=dev)
             res = {}
             for tag, w0 in (("bifocal", c["w0"]), ("plain", c["L"])):
                 reps = 3 if c["L"] > 8192 else 200
                 ms = time_calls(lambda: jl.jl_bifocal_prefill(q2, k2, v2, o2, l2, w0=w0, w_pretrained=c["W"],
-                                                              rope_base=c["base"], dev_error=err, stream=stream),
-                                reps)
+                                                              rope_base=c["base"], workspace=w2, dev_error=err,
+                                                              stream=stream), reps)
                 f = prefill_flop(c)
                 res[tag] = {"ms": round(ms, 4), "tflops": round(f / (ms * 1e-3) / 1e12, 2),
                             "tokens_per_s": round(c["B"] * c["L"] / (ms * 1e-3), 1)}
             res["shape"] = {k_: c[k_] for k_ in ("B", "L", "Hq", "Hkv", "D", "W", "w0", "base")}
             others[c["workload"]] = res
-            del q2, k2, v2, o2, l2
+            del q2, k2, v2, o2, l2, w2
         sweep = []
         sh = dict(B=1, Hq=32, Hkv=8, D=128, W=32768, base=1e6)
         dws1 = torch.zeros(jl.jl_decode_workspace_bytes(1, max(SWEEP_L), 32, 8, 128), dtype=torch.uint8, device=dev)
@@ -463,10 +467,12 @@ def run_ours(args):
             l2 = torch.empty(1, 32, L, dtype=torch.float32, device=dev)
             qd1, od1 = q2[:, L - 1].contiguous(), torch.empty(1, 32, 128, dtype=torch.bfloat16, device=dev)
             ld1 = torch.empty(1, 32, dtype=torch.float32, device=dev)
+            w2 = torch.empty(jl.jl_prefill_workspace_bytes(1, L, 32, 8, 128), dtype=torch.uint8, device=dev)
             for w0 in (0, 4096, L):
                 c = dict(sh, L=L, w0=w0)
                 pms = time_calls(lambda: jl.jl_bifocal_prefill(q2, k2, v2, o2, l2, w0=w0, w_pretrained=sh["W"],
-                                                               rope_base=sh["base"], dev_error=err, stream=stream), 2)
+                                                               rope_base=sh["base"], workspace=w2, dev_error=err,
+                                                               stream=stream), 2)
                 dms = time_calls(lambda: jl.jl_bifocal_decode(qd1, k2, v2, od1, ld1, L=L, w0=w0,
                                                               w_pretrained=sh["W"], rope_base=sh["base"],
                                                               workspace=dws1, dev_error=err, stream=stream), 20)
@@ -475,7 +481,7 @@ def run_ours(args):
                               "prefill_tokens_per_s": round(L / (pms * 1e-3), 1),
                               "decode_ms": round(dms, 4), "decode_gbs": round(decode_bytes(c) / (dms * 1e-3) / 1e9, 1),
                               "decode_tokens_per_s": round(1 / (dms * 1e-3), 1)})
-            del q2, k2, v2, o2, l2
+            del q2, k2, v2, o2, l2, w2
         others["length / band sweep (qwen3-4b shape, 1% x8 key outliers, decode B 1)"] = sweep
         del dws1
         if int(err.item()) != 0:
@@ -500,7 +506,7 @@ def run_ours(args):
 
         def e2e_call(bq, bk, bv, bo):
             jl.jl_bifocal_prefill(bq, bk, bv, bo, lse, w0=P["w0"], w_pretrained=P["W"], rope_base=P["base"],
-                                  dev_error=err, stream=stream)
+                                  workspace=ws, dev_error=err, stream=stream)
 
         def pipelined(reps):
             ev = lambda: torch.cuda.Event()
@@ -592,8 +598,8 @@ def run_ours(args):
                         "attention_ms": round(attn_ms_max, 3), "tokens_per_s": round(world * P["L"] * P["B"] /
                                                                                      (pre_ms_max * 1e-3), 1),
                         "attention_tflops": round(attn_tflops, 2),
-                        "path": "default: corrections inside the kernel, remote scores Q_hi K_hi + Q_hi K_lo + "
-                                "Q_lo K_hi (fp16 hi + lo), no workspace"},
+                        "path": "default: remote scores Q_hi K_hi + Q_hi K_lo + Q_lo K_hi (fp16 hi + lo); query "
+                                "block corrected inside the attention kernel, key rows by the correction pass"},
             "decode": {"value": dloop8["gbs_all_ranks"], "unit": "GB/s", "ms": dloop8["ms"],
                        "tokens_per_s": dloop8["tokens_per_s"], "B": Dc["B"],
                        "timing": f"{dloop8['reps']} launches back to back between two CUDA events, mean period",
@@ -621,7 +627,7 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": tensor_peak,
                          "unit": "TFLOP/s", "frac": round(attn_tflops / tensor_peak, 4),
                          "traffic": traffic.get("prefill_attention", {}).get("bytes_per_launch"),
-                         "kernel": "bifocal_prefill_hilo_kernel<128, true, 0>",
+                         "kernel": "bifocal_prefill_hilo_kernel<128, false, 0>",
                          "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a multi-second loop)",
                          "executed_tflops": round(exec_flop / (attn_ms_max * 1e-3) / 1e12, 2),
                          "executed_frac": round(exec_flop / (attn_ms_max * 1e-3) / 1e12 / tensor_peak, 4),
@@ -631,7 +637,7 @@ def run_ours(args):
                                      "peak_tflops_per_sm_ghz": round(tensor_peak / peak_ghz, 1) if peak_ghz else None,
                                      "note": "TFLOP/s divided by the median SM clock sampled while each ran"}},
             "e2e": e2e,
-            "gpu_launches": K * 2,
+            "gpu_launches": K * 3,
             "gpu_launches_decode_loops": dloop8["reps"] + dloop1["reps"],
             "clocks": clk,
             "cpu_baseline": cpu,

@@ -37,9 +37,10 @@
  *     memory and never writes its inputs.
  *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = default
  *     stream).  The return value reports argument checks and launch errors.
- *     Device-side failures (a pipeline wait that ran out of time) are written
- *     to *dev_error (a device int, may be NULL) as a non-zero value; the
- *     outputs are then invalid.
+ *     Device-side failures are written to *dev_error (a device int, may be
+ *     NULL) as a non-zero value -- 1: a pipeline wait ran out of time; 2: a
+ *     varlen sequence length out of range; 3: a corrected prefill operand
+ *     beyond fp16's range -- and the outputs are then invalid.
  *   - Reentrant; no global state beyond cached kernel attributes, with one
  *     exception: jl_bifocal_decode_noalloc keeps its scratch in a fixed device
  *     array inside the library, shared by every call on a device, so its
@@ -68,33 +69,36 @@ typedef enum {
 typedef enum { JL_QSHIFT_NONE = 0, JL_QSHIFT_SELF_EXTEND = 1 } jl_qshift;
 
 /*
- * Optional prefill flags, OR-ed into `mode` (decode ignores them).  The default
- * prefill (neither flag) applies the correction rotations R(p_q(i) - i) and
- * R(f(j) - j) inside the attention kernel, in fp32 registers, to the query
- * block once and to every remote key tile as it streams through shared memory,
- * and forms remote scores from fp16 hi + lo operands: S = Q_hi K_hi + Q_hi K_lo
- * + Q_lo K_hi with x = hi + lo to about 22 significant bits, so a score's
- * rounding error is about 2^-21 |q| |k| (in fp32 accumulation).  It needs no
- * scratch memory.  Local (base RoPE) scores and P V use the bf16 inputs as
- * they are.  Corrected values must stay within fp16's range: a query or key
- * component of magnitude 46340 or more can overflow, which the kernel reports
- * as device error 3 (results invalid).
+ * Optional prefill flags, OR-ed into `mode` (decode ignores them).
  *
+ * The default prefill forms remote scores from fp16 hi + lo operands:
+ * S = Q_hi K_hi + Q_hi K_lo + Q_lo K_hi, with x = hi + lo to about 22
+ * significant bits, so a score's rounding error is about 2^-21 |q| |k| (in
+ * fp32 accumulation).  The correction rotations are computed in fp32 from fp64
+ * angles: R(p_q(i) - i) is applied to the query block inside the attention
+ * kernel, in registers, on its way into tensor memory; R(f(j) - j) is applied
+ * to the key rows once per KV head by a correction pass that writes their hi
+ * and lo parts to the workspace (it serves every query head of the KV head).
+ * Local (base RoPE) scores and P V use the bf16 inputs as they are.  Corrected
+ * values must stay within fp16's range: a query or key component of magnitude
+ * 46340 or more can overflow, which is reported as device error 3 (results
+ * invalid).
+ *
+ * JL_PREFILL_KEYS_IN_KERNEL: the same arithmetic, with the key tiles also
+ *   corrected inside the attention kernel (a rotation warpgroup, one tile
+ *   ahead of the tensor core): no workspace, but slower on B200 (every query
+ *   head's CTAs redo the rotation of the shared key tiles).
  * JL_PREFILL_FP16: a correction pass writes R(p_q(i) - i) Q_i and R(f(j) - j) K_j
- *   to the workspace, rounded once to fp16, and the attention kernel forms each
- *   remote score with one fp16 product (two query heads per CTA).  Faster, but
+ *   rounded once to fp16, and the attention kernel forms each remote score
+ *   with one fp16 product (two query heads per CTA).  About twice as fast, but
  *   a score's rounding error is about 2^-11 |q| |k|: on rows dominated by one
  *   key of large norm that shows in the LSE (1e-2 on the pages' outlier
- *   workload).  Needs jl_prefill_workspace_bytes(...) of scratch.
- * JL_PREFILL_PREROTATED_K: the default's hi + lo arithmetic, but the key rows'
- *   hi / lo parts come from a correction pass into the workspace instead of
- *   being rotated inside the attention kernel (for comparing the two designs;
- *   same results up to the order of fp32 operations).  Needs scratch.
+ *   workload, against 1e-3 for the default).
  * The two flags are exclusive.  When every pair is local (G = 1 or w0 >= L) no
  * operand is corrected and every mode runs plain causal RoPE attention on the
- * bf16 inputs.
+ * bf16 inputs (two query heads per CTA), needing no workspace.
  */
-enum { JL_PREFILL_FP16 = 4, JL_PREFILL_PREROTATED_K = 8 };
+enum { JL_PREFILL_FP16 = 4, JL_PREFILL_KEYS_IN_KERNEL = 8 };
 
 /* Human-readable name of a status code (static string). */
 const char* jl_status_string(int status);
@@ -132,11 +136,10 @@ int jl_remote_positions(int64_t L, int64_t w0, int64_t w_pretrained, int mode, i
 int jl_prefill_tile_classes(int64_t L, int64_t w0, int64_t w_pretrained, int64_t* counts_out);
 
 /*
- * Scratch bytes jl_bifocal_prefill may need: the larger of the two opt-in
- * modes' needs (JL_PREFILL_FP16: fp16 corrected query and key rows, 2 * B * L *
- * (Hq + Hkv) * D bytes; JL_PREFILL_PREROTATED_K: fp16 hi and lo key rows,
- * 4 * B * L * Hkv * D bytes; each plus alignment).  The default mode needs
- * none (pass NULL and 0).  0 on bad arguments.
+ * Scratch bytes jl_bifocal_prefill may need: the larger of the default's
+ * (fp16 hi and lo key rows, 4 * B * L * Hkv * D bytes) and JL_PREFILL_FP16's
+ * (fp16 corrected query and key rows, 2 * B * L * (Hq + Hkv) * D bytes), each
+ * plus alignment.  JL_PREFILL_KEYS_IN_KERNEL needs none.  0 on bad arguments.
  */
 size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim);
 
@@ -147,13 +150,13 @@ size_t jl_prefill_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim);
  *   w0: band width of exact base-RoPE scoring (i - j < w0); w0 >= L, or
  *   L <= w_pretrained (G = 1), gives plain causal RoPE attention.
  *   mode: query shift (jl_qshift) | optional prefill flag (see above).
- *   workspace: NULL / 0 for the default mode; with JL_PREFILL_FP16 or
- *   JL_PREFILL_PREROTATED_K device scratch of at least
- *   jl_prefill_workspace_bytes(...) bytes (contents on entry do not matter;
- *   overwritten).
- * Launches: the default mode one kernel (the fused tcgen05 attention kernel,
- * correcting Q and K itself); the opt-in modes jl_prefill_correction (one or
- * two correction-rotation kernels) and then the attention kernel.  *dev_error
+ *   workspace: device scratch of at least jl_prefill_workspace_bytes(...)
+ *   bytes (contents on entry do not matter; overwritten); may be NULL / 0 with
+ *   JL_PREFILL_KEYS_IN_KERNEL or when every pair is local.
+ * Launches: jl_prefill_correction (one correction-rotation kernel for the
+ * keys; with JL_PREFILL_FP16 one for the queries too; none with
+ * JL_PREFILL_KEYS_IN_KERNEL or when every pair is local), then
+ * jl_prefill_attention (the fused tcgen05 attention kernel).  *dev_error
  * receives 1 (a pipeline wait ran out) or 3 (a corrected value beyond fp16's
  * range).
  * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_ALIGNMENT,
@@ -166,25 +169,26 @@ int jl_bifocal_prefill(const void* q, const void* k, const void* v, void* o, flo
 
 /*
  * First stage of jl_bifocal_prefill, exposed so the two stages can be timed or
- * scheduled separately.  Default mode: nothing to do (launches nothing).
- * JL_PREFILL_FP16: writes R(p_q(i) - i) Q_i as fp16 [B, L, Hq, D] to the
- * workspace, followed (at offset round_up(2 * B * L * Hq * D, 256)) by
- * R(f(j) - j) K_j as fp16 [B, L, Hkv, D].  JL_PREFILL_PREROTATED_K: writes the
- * key rows as fp16 hi [B, L, Hkv, D] and, at offset round_up(2 * B * L * Hkv *
- * D, 256), lo.  Only rows that have a remote partner are written (queries
- * i >= w0, keys j < L - w0).  The correction identity is the additive
- * composition of RoPE rotations (gist.science summary, "§2 On-the-Fly
- * Correctie Rotatie").  Launches nothing when every pair is local.  Errors as
- * jl_bifocal_prefill.
+ * scheduled separately: the correction pass.  Default: writes R(f(j) - j) K_j
+ * to the workspace as fp16 hi [B, L, Hkv, D] and, at offset round_up(2 * B *
+ * L * Hkv * D, 256), lo (hi + lo carries about 22 significant bits).
+ * JL_PREFILL_FP16: writes R(p_q(i) - i) Q_i as fp16 [B, L, Hq, D], followed (at
+ * offset round_up(2 * B * L * Hq * D, 256)) by R(f(j) - j) K_j as fp16
+ * [B, L, Hkv, D].  JL_PREFILL_KEYS_IN_KERNEL: nothing to do.  Only rows that
+ * have a remote partner are written (queries i >= w0, keys j < L - w0).  The
+ * correction identity is the additive composition of RoPE rotations
+ * (gist.science summary, "§2 On-the-Fly Correctie Rotatie").  A rotated value
+ * beyond fp16's range sets *dev_error (a device int, may be NULL) to 3.
+ * Launches nothing when every pair is local.  Errors as jl_bifocal_prefill.
  */
 int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, int Hkv, int head_dim, int w0,
                           int w_pretrained, double rope_base, int mode, void* workspace, size_t workspace_bytes,
-                          void* stream);
+                          int* dev_error, void* stream);
 
 /*
  * Second stage of jl_bifocal_prefill: the fused tcgen05 attention kernel
- * (one launch), reading Q, K, V and, in the opt-in modes, the corrected rows
- * that jl_prefill_correction left in `workspace` (same w0 / w_pretrained /
+ * (one launch), reading Q, K, V and the corrected rows that
+ * jl_prefill_correction left in `workspace` (same w0 / w_pretrained /
  * rope_base / mode).  Errors as jl_bifocal_prefill.
  */
 int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
@@ -192,9 +196,9 @@ int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, f
                          int mode, const void* workspace, size_t workspace_bytes, int* dev_error, void* stream);
 
 /*
- * Scratch bytes jl_bifocal_prefill_chunk may need in the opt-in modes (as
+ * Scratch bytes jl_bifocal_prefill_chunk may need (as
  * jl_prefill_workspace_bytes, with chunk_len query rows and q_offset +
- * chunk_len key rows); the default mode needs none.  0 on bad arguments.
+ * chunk_len key rows).  0 on bad arguments.
  */
 size_t jl_prefill_chunk_workspace_bytes(int B, int q_offset, int chunk_len, int Hq, int Hkv, int head_dim);
 
@@ -208,9 +212,8 @@ size_t jl_prefill_chunk_workspace_bytes(int B, int q_offset, int chunk_len, int 
  *   k_cache / v_cache [B, cache_len, Hkv, D]: bf16 device, already holding the
  *   chunk's own keys and values; read only.  q_offset + chunk_len <= cache_len.
  *   o [B, chunk_len, Hq, D] bf16; lse [B, Hq, chunk_len] fp32 or NULL.
- *   workspace: NULL / 0 in the default mode, else
- *   jl_prefill_chunk_workspace_bytes(...) bytes.  Everything else as
- *   jl_bifocal_prefill.
+ *   workspace: jl_prefill_chunk_workspace_bytes(...) bytes (NULL / 0 with
+ *   JL_PREFILL_KEYS_IN_KERNEL).  Everything else as jl_bifocal_prefill.
  * Note: a cache built by earlier decode steps is not equivalent to re-running
  * prefill over the whole sequence (the keys were rotated once, at their base
  * positions, either way; the hidden states are not recomputed).
@@ -222,8 +225,9 @@ int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_c
                              size_t workspace_bytes, int* dev_error, void* stream);
 
 /*
- * Scratch bytes jl_bifocal_prefill_ie needs: three fp32 partial outputs
- * [B, L, Hq, D] and their LSEs [B, Hq, L] (`mode` does not change it).
+ * Scratch bytes jl_bifocal_prefill_ie needs: the corrected key rows (hi and
+ * lo, every row), three fp32 partial outputs [B, L, Hq, D] and their LSEs
+ * [B, Hq, L] (`mode` does not change it).
  */
 size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim, int mode);
 
@@ -233,15 +237,16 @@ size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim
  * Inclusie-Exclusie Attention Merge"): three attention calls — (A) the window
  * 0 <= i - j < w0 with base RoPE, (B) every causal pair with remote positions,
  * (C) the window with remote positions — each writing an fp32 output and an
- * fp32 LSE (the default mode's kernel: corrections in the kernel, hi + lo
- * remote operands; the prefill flags in `mode` are ignored), merged as
+ * fp32 LSE (the default prefill path: hi + lo remote operands; the prefill
+ * flags in `mode` are ignored), merged as
  * O = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C), W_X = exp(LSE_X - max
  * LSE).  Same arguments and result as jl_bifocal_prefill up to rounding, which
  * the subtraction amplifies by (W_A + W_B + W_C) / (W_A + W_B - W_C): without
  * bound on rows where one key inside the window dominates both B and C.
  * workspace: jl_prefill_ie_workspace_bytes(...).  When every pair is local it
  * runs jl_bifocal_prefill.
- * Launches: three attention kernels and one merge kernel.
+ * Launches: one correction kernel (every key row), three attention kernels
+ * and one merge kernel.
  */
 int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
                           int Hkv, int head_dim, int w0, int w_pretrained, double rope_base, float softmax_scale,

@@ -72,8 +72,8 @@ constexpr int kMaxGridYZ = 65535;  // CUDA's limit on a grid's y and z dimension
 int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained, double rope_base, int mode) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || w0 < 0 || w_pretrained < 1) return JL_ERR_INVALID_ARG;
   if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return JL_ERR_INVALID_ARG;
-  if ((mode & ~(JL_QSHIFT_SELF_EXTEND | JL_PREFILL_FP16 | JL_PREFILL_PREROTATED_K)) != 0) return JL_ERR_INVALID_ARG;
-  if ((mode & JL_PREFILL_FP16) && (mode & JL_PREFILL_PREROTATED_K)) return JL_ERR_INVALID_ARG;
+  if ((mode & ~(JL_QSHIFT_SELF_EXTEND | JL_PREFILL_FP16 | JL_PREFILL_KEYS_IN_KERNEL)) != 0) return JL_ERR_INVALID_ARG;
+  if ((mode & JL_PREFILL_FP16) && (mode & JL_PREFILL_KEYS_IN_KERNEL)) return JL_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
   if (L > (1 << 30)) return JL_ERR_UNSUPPORTED;
@@ -201,11 +201,11 @@ int jl_prefill_tile_classes(int64_t L, int64_t w0, int64_t w_pretrained, int64_t
 
 namespace {
 
-// Prefill scratch (only the opt-in modes use any):
+// Prefill scratch:
+//   default                   corrected key rows as fp16 hi [B, Lk, Hkv, D], then lo
 //   JL_PREFILL_FP16           fp16 corrected query rows [B, Lq, Hq, D], then fp16
 //                             corrected key rows [B, Lk, Hkv, D]
-//   JL_PREFILL_PREROTATED_K   corrected key rows as fp16 hi [B, Lk, Hkv, D], then lo
-// The default mode corrects both sides inside the attention kernel and needs none.
+//   JL_PREFILL_KEYS_IN_KERNEL none (both sides corrected inside the attention kernel)
 size_t prefill_ws_fp16(int B, int Lq, int Lk, int Hq, int Hkv, int D) {
   return round_up((size_t)B * Lq * Hq * D * 2) + round_up((size_t)B * Lk * Hkv * D * 2);
 }
@@ -245,13 +245,13 @@ bool prefill_all_local(const PrefillProblem& pp, int w0, int w_pretrained) {
   return jl::all_local(pp.Lk(), w0, jl::group_size(pp.Lk(), w_pretrained));
 }
 
-// Scratch the call needs in this mode (0 for the default mode and whenever
-// every pair is local).
+// Scratch the call needs in this mode (0 with the keys corrected inside the
+// kernel and whenever every pair is local).
 size_t prefill_ws_need(const PrefillProblem& pp, int w0, int w_pretrained, int mode) {
   if (prefill_all_local(pp, w0, w_pretrained)) return 0;
   if (mode & JL_PREFILL_FP16) return prefill_ws_fp16(pp.B, pp.Lq, pp.Lk(), pp.Hq, pp.Hkv, pp.D);
-  if (mode & JL_PREFILL_PREROTATED_K) return prefill_ws_prerot(pp.B, pp.Lk(), pp.Hkv, pp.D);
-  return 0;
+  if (mode & JL_PREFILL_KEYS_IN_KERNEL) return 0;
+  return prefill_ws_prerot(pp.B, pp.Lk(), pp.Hkv, pp.D);
 }
 
 __half* ws_first(void* ws) { return reinterpret_cast<__half*>(ws); }
@@ -281,12 +281,14 @@ int workspace_checks(const PrefillProblem& pp, int w0, int w_pretrained, int mod
   return JL_OK;
 }
 
-// Correction pass of the opt-in modes (the default mode has none): fp16 rows
-// for JL_PREFILL_FP16, fp16 hi + lo key rows for JL_PREFILL_PREROTATED_K.
+// Correction pass: fp16 hi + lo key rows (default), fp16 query and key rows
+// (JL_PREFILL_FP16), nothing with JL_PREFILL_KEYS_IN_KERNEL.  all_keys: every
+// key row (the inclusion-exclusion call B scores every causal pair remotely),
+// not only those with a remote partner.
 int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double rope_base, int mode,
-                      void* workspace, cudaStream_t s) {
+                      void* workspace, int* dev_error, cudaStream_t s, bool all_keys = false) {
   if (prefill_all_local(pp, w0, w_pretrained)) return JL_OK;  // nothing to correct
-  if (!(mode & (JL_PREFILL_FP16 | JL_PREFILL_PREROTATED_K))) return JL_OK;
+  if (mode & JL_PREFILL_KEYS_IN_KERNEL) return JL_OK;
   const int64_t G = jl::group_size(pp.Lk(), w_pretrained);
   RotateArgs ra;
   std::memset(&ra, 0, sizeof(ra));
@@ -294,6 +296,7 @@ int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double
   ra.G = G;
   ra.shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
   ra.B = pp.B;
+  ra.dev_error = dev_error;
   const size_t kbytes = (size_t)pp.B * pp.Lk() * pp.Hkv * pp.D * 2;
   if (mode & JL_PREFILL_FP16) {
     // queries that have a remote key: positions q_off + r >= w0
@@ -322,7 +325,7 @@ int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double
   ra.H = pp.Hkv;
   ra.pos_off = 0;
   ra.row_begin = 0;
-  ra.row_end = pp.Lk() - w0;
+  ra.row_end = all_keys ? pp.Lk() : pp.Lk() - w0;
   ra.is_query = 0;
   if (jl::launch_rotate_rows(ra, pp.D, s) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
@@ -343,9 +346,10 @@ void fill_hilo_tables(jl::PrefillHiloArgs& a, int D, double rope_base) {
 // The attention launch.  Every pair local: the two-heads-per-CTA kernel on the
 // bf16 inputs (plain causal RoPE, no rounding of operands).  JL_PREFILL_FP16:
 // the same kernel on the fp16 rows of the correction pass.  Otherwise the hi +
-// lo kernel, correcting Q and K itself (or taking the key rows of
-// JL_PREFILL_PREROTATED_K from the workspace).  o_f32 (inclusion-exclusion
-// partials) writes fp32 instead of bf16 output.
+// lo kernel, correcting the query block itself and taking the key rows' hi /
+// lo parts from the workspace (or, with JL_PREFILL_KEYS_IN_KERNEL, correcting
+// the key tiles itself too).  o_f32 (inclusion-exclusion partials) writes fp32
+// instead of bf16 output.
 int attention_launch(const PrefillProblem& pp, void* o, float* o_f32, float* lse, int w0, int w_pretrained,
                      double rope_base, float softmax_scale, int mode, const void* workspace, int* dev_error,
                      cudaStream_t stream, int kind = jl::kBifocal) {
@@ -392,7 +396,7 @@ int attention_launch(const PrefillProblem& pp, void* o, float* o_f32, float* lse
     if (jl::launch_prefill(tq, tqr, tk, tkr, tv, pa, D, stream) != cudaSuccess) return JL_ERR_CUDA;
     return JL_OK;
   }
-  const bool rot_k = !(mode & JL_PREFILL_PREROTATED_K);
+  const bool rot_k = (mode & JL_PREFILL_KEYS_IN_KERNEL) != 0;
   CUtensorMap tkh = tk, tkl = tk;
   if (!rot_k) {
     void* ws = const_cast<void*>(workspace);
@@ -442,7 +446,7 @@ int prefill_entry(const PrefillProblem& pp, void* o, float* lse, int w0, int w_p
   if (st != JL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (correct) {
-    st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, s);
+    st = correction_launch(pp, w0, w_pretrained, rope_base, mode, workspace, dev_error, s);
     if (st != JL_OK) return st;
   }
   if (attend)
@@ -455,10 +459,10 @@ int prefill_entry(const PrefillProblem& pp, void* o, float* lse, int w0, int w_p
 
 int jl_prefill_correction(const void* q, const void* k, int B, int L, int Hq, int Hkv, int head_dim, int w0,
                           int w_pretrained, double rope_base, int mode, void* workspace, size_t workspace_bytes,
-                          void* stream) {
+                          int* dev_error, void* stream) {
   const PrefillProblem pp{q, k, k, B, 0, L, L, Hq, Hkv, head_dim};
   return prefill_entry(pp, nullptr, nullptr, w0, w_pretrained, rope_base, 0.f, mode, workspace, workspace_bytes,
-                       nullptr, stream, true, false);
+                       dev_error, stream, true, false);
 }
 
 int jl_prefill_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
@@ -491,11 +495,15 @@ int jl_bifocal_prefill_chunk(const void* q, const void* k_cache, const void* v_c
 namespace {
 
 struct IeLayout {
-  size_t o[3], lse[3], total;
+  size_t keys, o[3], lse[3], total;
 };
-IeLayout ie_layout(int B, int L, int Hq, int D) {
+// Corrected key rows (hi + lo, every row), then three fp32 partial outputs and
+// their LSEs.
+IeLayout ie_layout(int B, int L, int Hq, int Hkv, int D) {
   IeLayout lay;
   size_t off = 0;
+  lay.keys = off;
+  off += prefill_ws_prerot(B, L, Hkv, D);
   for (int x = 0; x < 3; ++x) {
     lay.o[x] = off;
     off += round_up((size_t)B * L * Hq * D * 4);
@@ -513,7 +521,7 @@ IeLayout ie_layout(int B, int L, int Hq, int D) {
 size_t jl_prefill_ie_workspace_bytes(int B, int L, int Hq, int Hkv, int head_dim, int mode) {
   (void)mode;
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || head_dim < 1) return 0;
-  return ie_layout(B, L, Hq, head_dim).total;
+  return ie_layout(B, L, Hq, Hkv, head_dim).total;
 }
 
 int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int Hq,
@@ -524,26 +532,28 @@ int jl_bifocal_prefill_ie(const void* q, const void* k, const void* v, void* o, 
   if (st != JL_OK) return st;
   if (!o) return JL_ERR_INVALID_ARG;
   if (!aligned16(o) || (lse && ((uintptr_t)lse & 3u))) return JL_ERR_ALIGNMENT;
-  const int qmode = mode & JL_QSHIFT_SELF_EXTEND;  // the three calls always correct in the kernel, hi + lo
+  const int qmode = mode & JL_QSHIFT_SELF_EXTEND;  // the three calls always use the default (hi + lo) path
   const int64_t G = jl::group_size(L, w_pretrained);
   if (jl::all_local(L, w0, G)) {
     // every pair local: the three calls collapse to plain causal attention
     return jl_bifocal_prefill(q, k, v, o, lse, B, L, Hq, Hkv, head_dim, w0, w_pretrained, rope_base, softmax_scale,
                               qmode, nullptr, 0, dev_error, stream);
   }
-  const IeLayout lay = ie_layout(B, L, Hq, head_dim);
+  const IeLayout lay = ie_layout(B, L, Hq, Hkv, head_dim);
   if (!workspace || workspace_bytes < lay.total) return JL_ERR_WORKSPACE;
   if (!aligned16(workspace)) return JL_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* ws = reinterpret_cast<char*>(workspace);
+  st = correction_launch(pp, w0, w_pretrained, rope_base, qmode, ws + lay.keys, dev_error, s, /*all_keys=*/true);
+  if (st != JL_OK) return st;
   const int kinds[3] = {jl::kWindowBase, jl::kCausalRemote, jl::kWindowRemote};
   jl::MergeArgs ma;
   std::memset(&ma, 0, sizeof(ma));
   for (int x = 0; x < 3; ++x) {
     float* ox = reinterpret_cast<float*>(ws + lay.o[x]);
     float* lx = reinterpret_cast<float*>(ws + lay.lse[x]);
-    st = attention_launch(pp, nullptr, ox, lx, w0, w_pretrained, rope_base, softmax_scale, qmode, nullptr, dev_error,
-                          s, kinds[x]);
+    st = attention_launch(pp, nullptr, ox, lx, w0, w_pretrained, rope_base, softmax_scale, qmode, ws + lay.keys,
+                          dev_error, s, kinds[x]);
     if (st != JL_OK) return st;
     ma.o_x[x] = ox;
     ma.lse_x[x] = lx;

@@ -19,6 +19,7 @@ struct RotateArgs {
   int row_begin, row_end;
   int is_query;      // 1: rotate by p_q(i) - i, 0: by f(j) - j
   int64_t G, shift;  // group size and query shift
+  int* dev_error;    // device int or null: set to kDevRange when a rotated value leaves fp16's range
   double theta[kMaxHalfDim];
 };
 cudaError_t launch_rotate_rows(const RotateArgs& args, int D, cudaStream_t stream);

@@ -1,6 +1,5 @@
-// Fused Dynamic Bifocal RoPE prefill for sm_100a, with the correction rotation
-// applied inside the kernel and remote scores carried at about 22 significant
-// bits.
+// Fused Dynamic Bifocal RoPE prefill for sm_100a, with remote scores carried at
+// about 22 significant bits (the library's default prefill path).
 //
 // A causal (query i, key j) pair with i - j < w0 is scored with the base-rotated
 // Q and K (exact base RoPE); every other causal pair with R(p_q(i)) q and
@@ -8,31 +7,37 @@
 // §1").  The inputs are rotated at their absolute positions, so the remote rows
 // are R(dq_i) Q_i and R(dk_j) K_j with dq_i = p_q(i) - i, dk_j = f(j) - j: RoPE
 // rotations compose additively (gist.science summary, "§2 On-the-Fly Correctie
-// Rotatie").  Nothing is written back to the inputs or to any scratch buffer:
-//   * a rotation warpgroup reads each key row of a remote tile from global
-//     memory one tile ahead, rotates it in fp32 registers and writes it into
-//     shared memory as fp16 hi + lo (hi = fp16(x), lo = fp16(x - hi)), in the
-//     128-byte-swizzled K-major layout the tensor core reads;
-//   * the same warpgroup rotates the block's query rows once into TMEM
-//     (Q_hi and Q_lo, the A operands);
+// Rotatie").  Nothing is written back to the inputs:
+//   * a rotation warpgroup rotates the block's query rows once, in fp32
+//     registers, into TMEM as fp16 hi + lo (hi = fp16(x), lo = fp16(x - hi);
+//     Q_hi and Q_lo are the A operands);
+//   * the key tiles' hi / lo rows come either from the correction pass
+//     (rope_rotate.cu, once per KV head, fp32 math; the default, kRotK =
+//     false) or from the same warpgroup, which then reads each key row of a
+//     remote tile from global memory one tile ahead, rotates it in registers
+//     and writes hi / lo into shared memory in the 128-byte-swizzled K-major
+//     layout the tensor core reads (kRotK = true; no scratch, but measured
+//     about 3x slower on B200: the per-tile row loads, the second unrolled
+//     code region and the per-tile synchronisation cost more than the
+//     correction pass, which serves every query head of a KV head at once);
 //   * a remote score tile is S = Q_hi K_hi + Q_hi K_lo + Q_lo K_hi (fp32
-//     accumulate): the operands carry about 22 significant bits, so a score's
-//     rounding error is about 2^-21 of |q| |k| instead of 2^-11 for one fp16
-//     product (which is what a key of large norm that dominates a softmax row
-//     turns into an LSE error).
-// Correction angles theta_t * dk come from a per-tile factor R(theta_t (dk_j0 -
-// 16 a)) (fp64 sincos, one per (tile, t), times a fixed table) and a 16-entry
-// table R(-theta_t b), with dk_j = dk_j0 - (16 a + b) inside the tile.
+//     accumulate): a score's rounding error is about 2^-21 of |q| |k|
+//     instead of 2^-11 for one fp16 product (which is what a key of large norm
+//     that dominates a softmax row turns into an LSE error).
+// In-kernel correction angles theta_t * d come from a factor R(theta_t (d_x0 -
+// 16 a)) for the row set's first row x0 (fp64: one sincos per CTA, then an
+// fp64 recurrence from one key tile to the next) times a table R(-theta_t b),
+// with d = d_x0 - (16 a + b) inside the set.
 //
 // Each 128 x 128 (query block, key block) tile is visited once per score set it
 // needs (remote passes first, then local passes; a tile straddling the band
 // edge gets both, with complementary masks), all feeding one online softmax.
 //
 // CTA = one 128-row query block of one query head.  Warp roles (384 threads):
-//   warp 0      TMA producer: V (2 stages); K (pre-rotated variant only)
+//   warp 0      TMA producer: V and (pre-rotated) K, 2 stages each
 //   warp 1      tcgen05 MMA issuer; owns the TMEM allocation (512 columns)
 //   warps 4-7   softmax (thread = query row = TMEM lane)
-//   warps 8-11  rotation: query rows into TMEM, key tiles into shared memory
+//   warps 8-11  rotation: query rows into TMEM (and key tiles with kRotK)
 // TMEM columns: S double buffer at 0 / 128 (P, bf16, overwrites the first 64
 // columns of its S), O at 256, Q_hi (or the base Q) at 256 + D, Q_lo at
 // 256 + 3D/2.  MMA order S(0) S(1) PV(0) S(2) PV(1) S(3) ...: the tensor core
@@ -134,6 +139,17 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b,
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// 16-byte global load that does not allocate in L1: the key rows stream
+// through once per tile, and L1 (what shared memory leaves of it) is kept for
+// the softmax's spilled registers.
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -614,7 +630,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
       const uint4* s4 = reinterpret_cast<const uint4*>(src);
 #pragma unroll
       for (int w = 0; w < H2 / 4; ++w) {
-        const uint4 v = valid ? __ldg(s4 + w) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 v = valid ? ldg_stream(s4 + w) : make_uint4(0u, 0u, 0u, 0u);
         raw[4 * w] = v.x;
         raw[4 * w + 1] = v.y;
         raw[4 * w + 2] = v.z;
@@ -642,7 +658,6 @@ __global__ void __launch_bounds__(kHThreads, 1)
     fill_c(2, dq0);
     mbar_arrive(bar(hCReady));
     ok = mbar_wait(bar(hCReady), 0, abort_flag, args.dev_error);
-    int c_phase = 1;
 
     // Query operands of the first pass kind.
     if (ok && npass > 0) {
@@ -662,38 +677,81 @@ __global__ void __launch_bounds__(kHThreads, 1)
     }
 
     if (kRotK) {
-      // Key tiles, one ahead: the next tile's rows are loaded (and its factors
-      // formed) while the tensor core still reads the stage they will fill.
-      auto key_row = [&](int nb) -> const __nv_bfloat16* {
-        const int j = nb * 128 + e;
-        return args.k + (((size_t)b * args.k_rows + (j < args.k_rows ? j : 0)) * args.Hkv + kvh) * D;
-      };
-      auto prep = [&](int p) -> bool {
+      // Key tiles.  Each thread rotates key row e of a tile; the rows of the
+      // next two tiles are kept in flight in two register buffers, so a
+      // tile's loads overlap the rotation of the one before it.
+      auto load_k = [&](uint32_t (&dst)[H2], int p) {
         const HPass ps = hilo_pass<kKind>(sc, p);
-        load_row(key_row(ps.nb), ps.nb * 128 + e < args.k_rows);
+        const int j = ps.nb * 128 + e;
+        const bool valid = j < args.k_rows;
+        const uint4* s4 = reinterpret_cast<const uint4*>(
+            args.k + (((size_t)b * args.k_rows + (valid ? j : 0)) * args.Hkv + kvh) * D);
+#pragma unroll
+        for (int w = 0; w < H2 / 4; ++w) {
+          const uint4 v = valid ? ldg_stream(s4 + w) : make_uint4(0u, 0u, 0u, 0u);
+          dst[4 * w] = v.x;
+          dst[4 * w + 1] = v.y;
+          dst[4 * w + 2] = v.z;
+          dst[4 * w + 3] = v.w;
+        }
+      };
+      // Per-tile factor base R(theta_t dk_j0) for this thread's t, carried in
+      // fp64 from one remote tile to the next (key blocks descend by one:
+      // dk_j0 grows by 128 - ceil(128 / G) or 128 - floor(128 / G)); one fp64
+      // sincos for the first remote tile of the CTA.
+      constexpr int TPT = 256 / D;
+      constexpr int APT = 8 / TPT;
+      const int ft = e / TPT;
+      const int fa0 = (e % TPT) * APT;
+      const double th = args.theta[ft];
+      const int64_t s_lo = 128 - (128 + G - 1) / G;
+      double st_s[2], st_c[2];
+      sincos(th * (double)s_lo, &st_s[0], &st_c[0]);
+      sincos(th * (double)(s_lo + 1), &st_s[1], &st_c[1]);
+      double kb_c = 1.0, kb_s = 0.0;
+      int64_t prev_dk0 = 0;
+      bool have_base = false;
+      auto fill_k = [&](int p) {
+        const HPass ps = hilo_pass<kKind>(sc, p);
         if (ps.remote) {
           const int64_t j0 = (int64_t)ps.nb * 128;
-          fill_c(p & 1, j0 / G - j0);
+          const int64_t dk0 = j0 / G - j0;
+          if (!have_base) {
+            sincos(th * (double)dk0, &kb_s, &kb_c);
+            have_base = true;
+          } else {
+            const int i = (int)(dk0 - prev_dk0 - s_lo);  // 0 or 1
+            const double c = kb_c * st_c[i] - kb_s * st_s[i];
+            kb_s = kb_c * st_s[i] + kb_s * st_c[i];
+            kb_c = c;
+          }
+          prev_dk0 = dk0;
+          const float cb = (float)kb_c, sb = (float)kb_s;
+#pragma unroll
+          for (int jj = 0; jj < APT; ++jj) {
+            const float2 m = args.t16[ft * 8 + fa0 + jj];
+            Cs[(p & 1) * kCElems + ((ft >> 1) * 8 + fa0 + jj) * 2 + (ft & 1)] =
+                make_float2(cb * m.x - sb * m.y, cb * m.y + sb * m.x);
+          }
         }
-        mbar_arrive(bar(hCReady));
-        const bool w = mbar_wait(bar(hCReady), (uint32_t)c_phase & 1u, abort_flag, args.dev_error);
-        ++c_phase;
-        return w;
+        mbar_arrive(bar(hCReady));  // tile p's factors (if any) are written
       };
-      if (ok && npass > 0) ok = prep(0);
-      for (int p = 0; p < npass && ok; ++p) {
+      const uint32_t rowoff = (uint32_t)(e * 128);
+      const uint32_t sw = (uint32_t)(e & 7);
+      auto unit_addr = [&](uint32_t slot, int U) -> uint32_t {
+        return slot + (uint32_t)((U >> 3) * kSlab) + rowoff + ((((uint32_t)U & 7u) ^ sw) << 4);
+      };
+      // Rotate (or, for a local pass, copy) tile p from `src` into its stage.
+      auto process = [&](const uint32_t (&src)[H2], int p) -> bool {
         const int s = p & 1;
         const HPass ps = hilo_pass<kKind>(sc, p);
-        if (!(ok = mbar_wait(bar(hKEmpty + s), ((uint32_t)(p >> 1) & 1u) ^ 1u, abort_flag, args.dev_error))) break;
+        // every thread's factors for tile p, then the stage's previous reader
+        if (!mbar_wait(bar(hCReady), (uint32_t)(p + 1) & 1u, abort_flag, args.dev_error)) return false;
+        if (!mbar_wait(bar(hKEmpty + s), ((uint32_t)(p >> 1) & 1u) ^ 1u, abort_flag, args.dev_error)) return false;
         const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
-        const uint32_t rowoff = (uint32_t)(e * 128);
-        const uint32_t sw = (uint32_t)(e & 7);
-        auto unit_addr = [&](uint32_t slot, int U) -> uint32_t {
-          return slot + (uint32_t)((U >> 3) * kSlab) + rowoff + ((((uint32_t)U & 7u) ^ sw) << 4);
-        };
         if (ps.remote) {
           const int64_t j0 = (int64_t)ps.nb * 128;
-          rotate_row_hilo<D>(raw, Cs + (p & 1) * kCElems, T1s, delta_of(j0), range,
+          rotate_row_hilo<D>(src, Cs + (p & 1) * kCElems, T1s, delta_of(j0), range,
                              [&](int U, const uint32_t (&h)[4], const uint32_t (&l)[4]) {
                                sts128(unit_addr(khi, U), h[0], h[1], h[2], h[3]);
                                sts128(unit_addr(khi + C::kTile, U), l[0], l[1], l[2], l[3]);
@@ -701,19 +759,40 @@ __global__ void __launch_bounds__(kHThreads, 1)
         } else {
 #pragma unroll
           for (int U = 0; U < D / 8; ++U)
-            sts128(unit_addr(khi, U), raw[4 * U], raw[4 * U + 1], raw[4 * U + 2], raw[4 * U + 3]);
+            sts128(unit_addr(khi, U), src[4 * U], src[4 * U + 1], src[4 * U + 2], src[4 * U + 3]);
         }
         fence_proxy_async_smem();  // the tensor core reads these rows through the async proxy
         mbar_arrive(bar(hKFull + s));
         if (q_switch && p == p_switch) {
           // The remote query operands have been read for the last time: put
           // the base rows in their place.
-          if (!(ok = mbar_wait(bar(hQEmpty), 0, abort_flag, args.dev_error))) break;
+          if (!mbar_wait(bar(hQEmpty), 0, abort_flag, args.dev_error)) return false;
           tc_fence_after();
-          load_row(qrow, qi < args.Lq);
-          write_base_q();
+          const uint4* q4 = reinterpret_cast<const uint4*>(qrow);
+#pragma unroll
+          for (int U = 0; U < D / 8; ++U) {
+            const uint4 w = qi < args.Lq ? ldg_stream(q4 + U) : make_uint4(0u, 0u, 0u, 0u);
+            tmem_st4(tmem + lane_off + kColQA + 4 * U, w.x, w.y, w.z, w.w);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(hQReady));
         }
-        if (p + 1 < npass && !(ok = prep(p + 1))) break;
+        if (p + 1 < npass) fill_k(p + 1);
+        return true;
+      };
+      uint32_t rawB[H2];
+      if (ok && npass > 0) {
+        load_k(raw, 0);
+        fill_k(0);
+        if (npass > 1) load_k(rawB, 1);
+      }
+      for (int p = 0; p < npass && ok; p += 2) {
+        if (!(ok = process(raw, p))) break;
+        if (p + 2 < npass) load_k(raw, p + 2);
+        if (p + 1 >= npass) break;
+        if (!(ok = process(rawB, p + 1))) break;
+        if (p + 3 < npass) load_k(rawB, p + 3);
       }
     } else if (ok && q_switch) {
       ok = mbar_wait(bar(hQEmpty), 0, abort_flag, args.dev_error);
@@ -753,15 +832,15 @@ cudaError_t launch_hilo_t(const CUtensorMap& tm_k, const CUtensorMap& tm_v, cons
 template <int D>
 cudaError_t launch_hilo_d(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_kh,
                           const CUtensorMap& tm_kl, const PrefillHiloArgs& a, bool rot_k, cudaStream_t stream) {
-  if (!rot_k) {
+  if (rot_k) {
     if (a.kind != kBifocal) return cudaErrorInvalidValue;
-    return launch_hilo_t<D, false, kBifocal>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    return launch_hilo_t<D, true, kBifocal>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
   }
   switch (a.kind) {
-    case kWindowBase: return launch_hilo_t<D, true, kWindowBase>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
-    case kCausalRemote: return launch_hilo_t<D, true, kCausalRemote>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
-    case kWindowRemote: return launch_hilo_t<D, true, kWindowRemote>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
-    default: return launch_hilo_t<D, true, kBifocal>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    case kWindowBase: return launch_hilo_t<D, false, kWindowBase>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    case kCausalRemote: return launch_hilo_t<D, false, kCausalRemote>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    case kWindowRemote: return launch_hilo_t<D, false, kWindowRemote>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
+    default: return launch_hilo_t<D, false, kBifocal>(tm_k, tm_v, tm_kh, tm_kl, a, stream);
   }
 }
 

@@ -10,10 +10,13 @@
 //
 // Angles reach ~1e5 rad at 128K tokens, so they are formed and reduced in fp64
 // (one sincos per (row, pair), shared by every head of the row); the rotation
-// itself is fp32 and the output is rounded to fp16 (round-to-nearest-even):
-// the rotated rows only feed the score product, and fp16 keeps three more
-// mantissa bits than bf16 at the same tensor-core rate (inputs are bounded by
-// fp16's range, |x| < 65504).
+// itself is fp32 and the output is rounded to fp16 (round-to-nearest-even),
+// optionally with the rounding residual as a second fp16 row (hi + lo carry
+// about 22 significant bits): the rotated rows only feed the score products,
+// and fp16 keeps three more mantissa bits than bf16 at the same tensor-core
+// rate.  A rotated value beyond fp16's range (|x| >= 65520, reachable from
+// inputs of magnitude 46340 or more) cannot be carried: the kernel reports it
+// as kDevRange in *dev_error, and the results are invalid.
 #include "jl_kernels.cuh"
 
 namespace jl {
@@ -50,6 +53,7 @@ __global__ void __launch_bounds__(kRotThreads)
 
   constexpr int kChunks = H2 / 8;  // 8 pairs (16 B of each half) per work item
   const int items = kRotRows * args.H * kChunks;
+  uint32_t range = 0;  // bit 15 / 31 set by an fp16 half that is inf or NaN
   for (int w = threadIdx.x; w < items; w += blockDim.x) {
     const int ch = w % kChunks;
     const int h = (w / kChunks) % args.H;
@@ -81,6 +85,9 @@ __global__ void __launch_bounds__(kRotThreads)
       lo_out[k] = pack_f16x2(rx[2 * k], rx[2 * k + 1]);
       hi_out[k] = pack_f16x2(ry[2 * k], ry[2 * k + 1]);
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      range |= ((lo_out[k] & 0x7FFF7FFFu) + 0x04000400u) | ((hi_out[k] & 0x7FFF7FFFu) + 0x04000400u);
     *reinterpret_cast<uint4*>(args.y + base + ch * 8) = make_uint4(lo_out[0], lo_out[1], lo_out[2], lo_out[3]);
     *reinterpret_cast<uint4*>(args.y + base + H2 + ch * 8) =
         make_uint4(hi_out[0], hi_out[1], hi_out[2], hi_out[3]);
@@ -98,6 +105,7 @@ __global__ void __launch_bounds__(kRotThreads)
       *reinterpret_cast<uint4*>(args.y_lo + base + H2 + ch * 8) = make_uint4(rh[0], rh[1], rh[2], rh[3]);
     }
   }
+  if ((range & 0x80008000u) != 0u && args.dev_error != nullptr) atomicExch(args.dev_error, kDevRange);
 }
 
 }  // namespace

@@ -14,7 +14,7 @@ import os
 import numpy as np
 
 __all__ = [
-    "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JL_PREFILL_FP16", "JL_PREFILL_PREROTATED_K", "JetLongError", "lib", "library_path",
+    "JL_QSHIFT_NONE", "JL_QSHIFT_SELF_EXTEND", "JL_PREFILL_FP16", "JL_PREFILL_KEYS_IN_KERNEL", "JetLongError", "lib", "library_path",
     "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes", "jl_decode_workspace_bytes",
     "jl_bifocal_prefill", "jl_bifocal_decode", "jl_prefill_correction", "jl_prefill_attention",
     "jl_bifocal_decode_noalloc", "jl_bifocal_decode_varlen", "jl_rope_append", "jl_prefill_chunk_workspace_bytes",
@@ -25,11 +25,11 @@ __all__ = [
 
 JL_QSHIFT_NONE = 0
 JL_QSHIFT_SELF_EXTEND = 1
-# Optional prefill flags OR-ed into mode (include/jl_api.h): the default corrects Q
-# and K inside the attention kernel with fp16 hi + lo remote operands and needs no
-# workspace.
-JL_PREFILL_FP16 = 4          # one fp16 product per remote score from pre-rotated rows (needs workspace)
-JL_PREFILL_PREROTATED_K = 8  # default arithmetic, key rows' hi / lo from a correction pass (needs workspace)
+# Optional prefill flags OR-ed into mode (include/jl_api.h).  The default carries
+# remote scores as fp16 hi + lo products: query rows corrected inside the attention
+# kernel, key rows by a correction pass into the workspace.
+JL_PREFILL_FP16 = 4            # one fp16 product per remote score from pre-rotated rows (workspace)
+JL_PREFILL_KEYS_IN_KERNEL = 8  # default arithmetic, key tiles corrected inside the kernel too (no workspace)
 EXPORTED_SYMBOLS = (
     "jl_status_string", "jl_group_size", "jl_remote_positions", "jl_prefill_workspace_bytes",
     "jl_bifocal_prefill", "jl_decode_workspace_bytes", "jl_bifocal_decode", "jl_prefill_correction",
@@ -75,7 +75,7 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_prefill.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_f, c_i,
                                      c_p, c_sz, c_p, c_p]
     L.jl_bifocal_prefill.restype = c_i
-    L.jl_prefill_correction.argtypes = [c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_i, c_p, c_sz, c_p]
+    L.jl_prefill_correction.argtypes = [c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_i, c_p, c_sz, c_p, c_p]
     L.jl_prefill_correction.restype = c_i
     L.jl_prefill_attention.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_f, c_i,
                                        c_p, c_sz, c_p, c_p]
@@ -174,9 +174,9 @@ def jl_bifocal_prefill(q, k, v, o, lse, *, w0: int, w_pretrained: int, rope_base
                        softmax_scale: float = 0.0, mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None,
                        dev_error=None, stream=None):
     """Fused bifocal prefill.  q [B, L, Hq, D], k / v [B, L, Hkv, D], o like q (bf16, CUDA);
-    lse [B, Hq, L] fp32 or None; workspace: None in the default mode, else a uint8 CUDA
-    tensor of jl_prefill_workspace_bytes(...) bytes (JL_PREFILL_FP16 /
-    JL_PREFILL_PREROTATED_K)."""
+    lse [B, Hq, L] fp32 or None; workspace: a uint8 CUDA tensor of
+    jl_prefill_workspace_bytes(...) bytes (None with JL_PREFILL_KEYS_IN_KERNEL, or when
+    every pair is local)."""
     import torch
     B, L, Hq, D = q.shape
     Hkv = k.shape[2]
@@ -194,7 +194,7 @@ def jl_bifocal_prefill(q, k, v, o, lse, *, w0: int, w_pretrained: int, rope_base
 
 
 def jl_prefill_correction(q, k, *, w0: int, w_pretrained: int, rope_base: float,
-                          mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None, stream=None):
+                          mode: int = JL_QSHIFT_SELF_EXTEND, workspace=None, dev_error=None, stream=None):
     """Stage 1 of jl_bifocal_prefill: corrected Q / K rows into the workspace."""
     import torch
     B, L, Hq, D = q.shape
@@ -203,7 +203,8 @@ def jl_prefill_correction(q, k, *, w0: int, w_pretrained: int, rope_base: float,
     _check_tensor(k, "k", torch.bfloat16, (B, L, Hkv, D))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().jl_prefill_correction(_ptr(q), _ptr(k), B, L, Hq, Hkv, D, int(w0), int(w_pretrained),
-                                     float(rope_base), int(mode), _ptr(workspace), ws_bytes, _stream(stream))
+                                     float(rope_base), int(mode), _ptr(workspace), ws_bytes, _ptr(dev_error),
+                                     _stream(stream))
     _check(st, "jl_prefill_correction")
 
 

@@ -17,15 +17,16 @@ O_MEAN_ABS = 2e-3
 LSE_MAX_ABS = 1e-3
 
 MODES = {jo.MODE_NONE: jl.JL_QSHIFT_NONE, jo.MODE_SELF_EXTEND: jl.JL_QSHIFT_SELF_EXTEND}
-# Prefill variants: the default (corrections inside the attention kernel, hi + lo
-# remote operands), the same arithmetic with key rows pre-rotated by a correction
-# pass, and the opt-in single-fp16-product path.
-PRECISIONS = {"default": 0, "prerot": jl.JL_PREFILL_PREROTATED_K, "fp16": jl.JL_PREFILL_FP16}
+# Prefill variants: the default (hi + lo remote operands; query rows corrected in
+# the attention kernel, key rows by a correction pass), the same arithmetic with
+# the key tiles corrected inside the kernel too, and the opt-in single-fp16-product
+# path.
+PRECISIONS = {"default": 0, "inkernel": jl.JL_PREFILL_KEYS_IN_KERNEL, "fp16": jl.JL_PREFILL_FP16}
 
 
 def prefill_workspace(prec, nbytes, dev):
-    """Scratch for a prefill variant (None for the default, which needs none)."""
-    return None if PRECISIONS[prec] == 0 else torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    """Scratch for a prefill variant (None when the key tiles are corrected in the kernel)."""
+    return None if prec == "inkernel" else torch.empty(nbytes, dtype=torch.uint8, device=dev)
 
 
 def run_prefill(q, k, v, *, w0, W, base, mode=jo.MODE_SELF_EXTEND, scale=0.0, prec="default"):

@@ -41,16 +41,15 @@ def _margins_intact(raw, what):
     assert bool((raw[-PAD:] == FILL).all()), f"{what}: write past the buffer"
 
 
-@pytest.mark.parametrize("prec", ["default", "prerot", "fp16"])
+@pytest.mark.parametrize("prec", ["default", "inkernel", "fp16"])
 def test_prefill_writes_only_its_outputs(prec):
-    # (the default mode takes no workspace; the opt-in modes' workspace is
-    # checked like the outputs)
+    # (the workspace, where the mode takes one, is checked like the outputs)
     B, L, Hq, Hkv, D, W, w0 = 2, 700, 4, 2, 128, 200, 150
     q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=31, outlier_frac=0.01)
     qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
     q0, k0, v0 = qd.clone(), kd.clone(), vd.clone()
     mode = jl.JL_QSHIFT_SELF_EXTEND | PRECISIONS[prec]
-    ws_bytes = jl.jl_prefill_workspace_bytes(B, L, Hq, Hkv, D) if PRECISIONS[prec] else 0
+    ws_bytes = 0 if prec == "inkernel" else jl.jl_prefill_workspace_bytes(B, L, Hq, Hkv, D)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
 
     o_raw, o = _padded((B, L, Hq, D), torch.bfloat16)
@@ -115,18 +114,17 @@ def test_chunked_prefill_writes_only_its_outputs():
     l_raw, lse = _padded((B, Hq, C), torch.float32)
     w_raw, ws = _padded((ws_bytes,), torch.uint8)
     jl.jl_bifocal_prefill_chunk(qd, kd, vd, o, lse, q_offset=P, w0=w0, w_pretrained=W, rope_base=1e6,
-                                mode=jl.JL_QSHIFT_SELF_EXTEND | jl.JL_PREFILL_PREROTATED_K, workspace=ws,
-                                dev_error=err)
+                                workspace=ws, dev_error=err)
     torch.cuda.synchronize()
     for raw, what in ((o_raw, "O"), (l_raw, "LSE"), (w_raw, "workspace")):
         _margins_intact(raw, what)
     assert torch.equal(kd, k0) and torch.equal(vd, v0), "cache was written"
-    # the default mode (no workspace) on the same chunk: same outputs within
-    # rounding, margins intact
+    # the key tiles corrected in the kernel (no workspace) on the same chunk:
+    # same outputs within rounding, margins intact
     o3_raw, o3 = _padded((B, C, Hq, D), torch.bfloat16)
     l3_raw, lse3 = _padded((B, Hq, C), torch.float32)
     jl.jl_bifocal_prefill_chunk(qd, kd, vd, o3, lse3, q_offset=P, w0=w0, w_pretrained=W, rope_base=1e6,
-                                dev_error=err)
+                                mode=jl.JL_QSHIFT_SELF_EXTEND | jl.JL_PREFILL_KEYS_IN_KERNEL, dev_error=err)
     torch.cuda.synchronize()
     _margins_intact(o3_raw, "O (default)")
     _margins_intact(l3_raw, "LSE (default)")

@@ -61,7 +61,7 @@ def _oracle_chunk(q_full, k, v, P, C, w0, W, base, mode=jo.MODE_SELF_EXTEND):
     (1111, 389, 0, 400, jo.MODE_SELF_EXTEND, "default", 0.01),   # w0 = 0: every pair remote
     (5, 50, 16, 20, jo.MODE_SELF_EXTEND, "default", 0.0),        # small chunk, stale rows after it in the cache
     (900, 600, 200, 1600, jo.MODE_SELF_EXTEND, "default", 0.0),  # G = 1 at the total length: plain causal RoPE
-    (700, 800, 200, 400, jo.MODE_SELF_EXTEND, "prerot", 0.01),   # key rows' hi / lo from the correction pass
+    (700, 800, 200, 400, jo.MODE_SELF_EXTEND, "inkernel", 0.01),  # key tiles corrected in the kernel
     (700, 800, 200, 400, jo.MODE_SELF_EXTEND, "fp16", 0.0),      # single fp16 product
 ])
 def test_chunk_matches_oracle(P, C, w0, W, mode, prec, outl):
@@ -81,7 +81,8 @@ def test_final_chunk_equals_whole_prefill_rows():
     qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
     o_full = torch.empty_like(qd)
     lse_full = torch.empty(1, 8, L, dtype=torch.float32, device=DEV)
-    jl.jl_bifocal_prefill(qd, kd, vd, o_full, lse_full, w0=w0, w_pretrained=W, rope_base=1e6)
+    ws = torch.empty(jl.jl_prefill_workspace_bytes(1, L, 8, 2, 128), dtype=torch.uint8, device=DEV)
+    jl.jl_bifocal_prefill(qd, kd, vd, o_full, lse_full, w0=w0, w_pretrained=W, rope_base=1e6, workspace=ws)
     kbig = torch.cat([kd, torch.full((1, 300, 2, 128), 7.0, dtype=torch.bfloat16, device=DEV)], dim=1)
     vbig = torch.cat([vd, torch.full((1, 300, 2, 128), -7.0, dtype=torch.bfloat16, device=DEV)], dim=1)
     o_c, lse_c = _chunk(qd[:, P:].contiguous(), kbig, vbig, P, w0, W, 1e6)

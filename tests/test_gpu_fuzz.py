@@ -46,7 +46,7 @@ def _prefill_cases(n=40, seed=2024):
         D, Hq, Hkv, W, w0, mode = _draw(rng, L)
         B = int(rng.integers(1, 3))
         u = rng.random()
-        prec = "prerot" if u < 0.2 else ("fp16" if u < 0.35 else "default")
+        prec = "inkernel" if u < 0.2 else ("fp16" if u < 0.35 else "default")
         outl = 0.0 if prec == "fp16" else float(rng.choice([0.0, 0.01]))
         cases.append((B, L, Hq, Hkv, D, W, w0, mode, prec, outl))
     return cases
@@ -104,9 +104,10 @@ def test_chunked_prefill_random_shapes(P, C, Hq, Hkv, D, W, w0, mode):
     kd, vd = k.to(DEV), v.to(DEV)
     o = torch.empty_like(q)
     lse = torch.empty(1, Hq, C, dtype=torch.float32, device=DEV)
+    ws = torch.empty(jl.jl_prefill_chunk_workspace_bytes(1, P, C, Hq, Hkv, D), dtype=torch.uint8, device=DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
     jl.jl_bifocal_prefill_chunk(q, kd, vd, o, lse, q_offset=P, w0=w0, w_pretrained=W, rope_base=10000.0,
-                                mode=MODES[mode], dev_error=err)
+                                mode=MODES[mode], workspace=ws, dev_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     p = jo.BifocalParams(L=P + C, w0=w0, w_pretrained=W, base=10000.0, mode=mode)

@@ -92,10 +92,12 @@ def test_prefill_graph_replay_matches_eager():
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     o = torch.empty_like(qd)
     lse = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    ws = torch.empty(jl.jl_prefill_workspace_bytes(B, L, Hq, Hkv, D), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def call():
-        jl.jl_bifocal_prefill(qd, kd, vd, o, lse, w0=w0, w_pretrained=W, rope_base=1e6, dev_error=err)
+        jl.jl_bifocal_prefill(qd, kd, vd, o, lse, w0=w0, w_pretrained=W, rope_base=1e6, workspace=ws,
+                              dev_error=err)
 
     call()
     torch.cuda.synchronize()

@@ -60,7 +60,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("prec", ["default", "prerot", "fp16"])
+@pytest.mark.parametrize("prec", ["default", "inkernel", "fp16"])
 @pytest.mark.parametrize("B,L,Hq,Hkv,D,W,w0,mode,outl", CASES)
 def test_prefill_small_cases(B, L, Hq, Hkv, D, W, w0, mode, outl, prec):
     if prec == "fp16" and outl > 0.0:
@@ -237,14 +237,15 @@ SWEEP_HEADS = [0, 3, 6, 13, 17, 22, 28, 31]  # 8 of 32 query heads, every KV hea
 def test_prefill_sweep_sampled(L):
     # Qwen3-4B shape with 1% x8 outlier keys, w0 in {0, 4096, L}: >= 64 random
     # rows (plus band and tile edges) on 8 heads, for the default and the
-    # pre-rotated-key variant, against the same oracle rows.
+    # variant that corrects the key tiles inside the kernel, against the same
+    # oracle rows.
     W = 32768
     q, k, v = synthetic.prefill_inputs(1, L, 32, 8, 128, seed=L, outlier_frac=0.01)
     for w0 in (0, 4096, L):
         rows = sample_rows(L, w0, 64, seed=w0)
         p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
         ref = oracle_prefill_rows(q, k, v, rows, SWEEP_HEADS, p)
-        for prec in ("default", "prerot"):
+        for prec in ("default", "inkernel"):
             o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6, prec=prec)
             assert err == 0
             for h in SWEEP_HEADS:
@@ -283,11 +284,11 @@ def test_prefill_outlier_dominated_rows_128k():
     assert checked >= 192
 
 
-def test_prefill_prerotated_keys_full_size_sampled():
-    # the Qwen3-8B-shaped 128K workload through the pre-rotated-key variant
+def test_prefill_keys_in_kernel_full_size_sampled():
+    # the Qwen3-8B-shaped 128K workload with the key tiles corrected in the kernel
     L, W, w0 = 131072, 32768, 4096
     q, k, v = synthetic.prefill_inputs(1, L, 32, 8, 128, seed=0)
-    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6, prec="prerot")
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=1e6, prec="inkernel")
     assert err == 0
     rows = sample_rows(L, w0, 256, seed=2)
     heads = [0, 17, 31]
@@ -295,10 +296,10 @@ def test_prefill_prerotated_keys_full_size_sampled():
     ref = oracle_prefill_rows(q, k, v, rows, heads, p)
     for h in heads:
         o_ref, lse_ref = ref[h]
-        assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref, f"prerot 128k h{h}")
+        assert_close(o[0, rows, h].numpy(), o_ref, lse[0, h, rows].numpy(), lse_ref, f"keys in kernel 128k h{h}")
 
 
-@pytest.mark.parametrize("prec", ["default", "prerot", "fp16"])
+@pytest.mark.parametrize("prec", ["default", "inkernel", "fp16"])
 def test_two_stage_prefill_equals_fused_call(prec):
     # jl_prefill_correction then jl_prefill_attention (the two stages the fused
     # entry point launches) give the same bits, and one correction pass serves
@@ -327,15 +328,15 @@ def test_two_stage_prefill_equals_fused_call(prec):
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_prefill_default_and_prerotated_keys_agree():
+def test_prefill_key_correction_pass_and_in_kernel_agree():
     # The two hi + lo variants differ only in where the key rows are rotated
-    # (registers inside the kernel, or a correction pass): both corrections
+    # (a correction pass, or registers inside the kernel): both corrections
     # are fp32 rotations by the same angles, so the outputs agree to within a
     # few units of bf16 rounding, and the LSEs to fp32 rounding.
     B, L, Hq, Hkv, D, W, w0 = 1, 2000, 8, 2, 128, 600, 300
     q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=21, outlier_frac=0.01)
     o1, l1, e1 = run_prefill(q, k, v, w0=w0, W=W, base=1e6)
-    o2, l2, e2 = run_prefill(q, k, v, w0=w0, W=W, base=1e6, prec="prerot")
+    o2, l2, e2 = run_prefill(q, k, v, w0=w0, W=W, base=1e6, prec="inkernel")
     assert e1 == 0 and e2 == 0
     assert (o1 - o2).abs().max().item() <= 1.6e-2
     assert (l1 - l2).abs().max().item() <= 2e-4

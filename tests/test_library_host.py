@@ -112,11 +112,11 @@ def test_remote_positions_rejects_bad_args(lib):
     assert lib.jl_remote_positions(10, 0, 10, 2, None, None) == JL_ERR_INVALID_ARG  # not a position-map mode
 
 
-FP16, PREROT = jl.JL_PREFILL_FP16, jl.JL_PREFILL_PREROTATED_K
+FP16, INKERNEL = jl.JL_PREFILL_FP16, jl.JL_PREFILL_KEYS_IN_KERNEL
 
 
 def test_workspace_sizes(lib):
-    # the larger of the two opt-in modes' needs (the default mode needs none)
+    # the larger of the default's (fp16 hi + lo key rows) and JL_PREFILL_FP16's needs
     assert jl.jl_prefill_workspace_bytes(1, 131072, 32, 8, 128) >= 2 * 131072 * (32 + 8) * 128
     assert jl.jl_prefill_workspace_bytes(1, 4096, 2, 2, 128) >= 4 * 4096 * 2 * 128
     assert jl.jl_prefill_workspace_bytes(0, 10, 1, 1, 64) == 0
@@ -154,13 +154,13 @@ def test_prefill_argument_errors(lib):
     assert _prefill(lib, base=0.0) == JL_ERR_INVALID_ARG
     assert _prefill(lib, mode=2) == JL_ERR_INVALID_ARG    # not a flag
     assert _prefill(lib, mode=16 | 1) == JL_ERR_INVALID_ARG
-    assert _prefill(lib, mode=FP16 | PREROT | 1) == JL_ERR_INVALID_ARG  # exclusive flags
-    # the opt-in modes need the workspace jl_prefill_workspace_bytes reports
-    # (every call below fails its checks, so nothing is launched on the fake
-    # addresses; the default mode needs no workspace, so its workspace
-    # arguments are never checked and are not exercised here)
+    assert _prefill(lib, mode=FP16 | INKERNEL | 1) == JL_ERR_INVALID_ARG  # exclusive flags
+    # the default and JL_PREFILL_FP16 need the workspace jl_prefill_workspace_bytes
+    # reports (every call below fails its checks, so nothing is launched on the
+    # fake addresses; JL_PREFILL_KEYS_IN_KERNEL needs no workspace, so its
+    # workspace arguments are never checked and are not exercised here)
     need = lib.jl_prefill_workspace_bytes(1, 256, 4, 2, 128)
-    for flag in (FP16, PREROT):
+    for flag in (0, FP16):
         assert _prefill(lib, mode=flag | 1, ws_bytes=need // 3) == JL_ERR_WORKSPACE
         assert _prefill(lib, mode=flag | 1, ws=None) == JL_ERR_WORKSPACE
         assert _prefill(lib, mode=flag | 1, ws=A + 4) == JL_ERR_ALIGNMENT
@@ -214,6 +214,7 @@ def test_prefill_chunk_argument_errors(lib):
     need = lib.jl_prefill_chunk_workspace_bytes(1, 100, 156, 4, 2, 128)
     assert need == jl.jl_prefill_chunk_workspace_bytes(1, 100, 156, 4, 2, 128) > 0
     assert chunk(ws_bytes=need - 1, mode=FP16 | 1) == JL_ERR_WORKSPACE
+    assert chunk(ws_bytes=need // 3) == JL_ERR_WORKSPACE
     # a whole-sequence chunk needs what jl_prefill_workspace_bytes reports
     assert lib.jl_prefill_chunk_workspace_bytes(2, 0, 300, 8, 2, 64) == lib.jl_prefill_workspace_bytes(2, 300, 8, 2, 64)
 
