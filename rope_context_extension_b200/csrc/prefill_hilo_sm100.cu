@@ -318,6 +318,15 @@ __global__ void __launch_bounds__(kHThreads, 1)
       const uint32_t id_loc = make_idesc_16bit(128, 128, false, false);  // bf16 Q K
       const uint32_t id_rem = make_idesc_16bit(128, 128, false, true);   // fp16 Q_hi / Q_lo, K_hi / K_lo
       const uint32_t id_pv = make_idesc_16bit(128, D, true, false);      // bf16 P V
+      // Shared-memory matrix descriptors, built once: K_hi of each stage (K_lo
+      // is one tile further) and V of each stage.  A k-step of 16 elements
+      // moves the start address by 32 B inside a 128-byte slab and by a slab
+      // every four steps; the address field holds bytes >> 4.
+      const uint64_t dk_hi0 = make_sdesc_sw128(sbase + C::kKOff, 16, 1024);
+      const uint64_t dk_hi1 = make_sdesc_sw128(sbase + C::kKOff + 2 * C::kTile, 16, 1024);
+      const uint64_t dv0 = make_sdesc_sw128(sbase + C::kVOff, kSlab, 1024);
+      const uint64_t dv1 = make_sdesc_sw128(sbase + C::kVOff + C::kTile, kSlab, 1024);
+      auto kstep_off = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * kSlab + (ks & 3) * 32) >> 4); };
       auto issue_s = [&](int p) -> bool {
         const int s = p & 1;
         const uint32_t ph = (uint32_t)(p >> 1) & 1u;
@@ -328,26 +337,22 @@ __global__ void __launch_bounds__(kHThreads, 1)
         tc_fence_after();
         const HPass ps = hilo_pass<kKind>(sc, p);
         const uint32_t d = tmem + (uint32_t)(128 * s);
-        const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
-        const uint32_t klo = khi + C::kTile;
+        // descriptors of the stage's K_hi / K_lo tiles (k-step offsets are
+        // added below as compile-time constants: one add per MMA)
+        const uint64_t dkh = s == 0 ? dk_hi0 : dk_hi1;
+        const uint64_t dkl = dkh + (uint64_t)(C::kTile >> 4);
         const uint32_t id_s = ps.remote ? id_rem : id_loc;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t o = (uint32_t)((ks >> 2) * kSlab + (ks & 3) * 32);
-          mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), make_sdesc_sw128(khi + o, 16, 1024), id_s, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_s, ks > 0 ? 1u : 0u);
         if (ps.remote) {
           // + Q_hi K_lo + Q_lo K_hi into the same accumulator
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t o = (uint32_t)((ks >> 2) * kSlab + (ks & 3) * 32);
-            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), make_sdesc_sw128(klo + o, 16, 1024), id_s, 1u);
-          }
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkl + kstep_off(ks), id_s, 1u);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t o = (uint32_t)((ks >> 2) * kSlab + (ks & 3) * 32);
-            mma_ts(d, tmem + kColQB + (uint32_t)(ks * 8), make_sdesc_sw128(khi + o, 16, 1024), id_s, 1u);
-          }
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ts(d, tmem + kColQB + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_s, 1u);
         }
         tc_commit(bar(hSFull + s));
         tc_commit(bar(hKEmpty + s));
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
         const int s = p & 1;
         const uint32_t ph = (uint32_t)(p >> 1) & 1u;
         if (!mbar_wait(bar(hVFull + s), ph, abort_flag, args.dev_error)) return false;
-        const uint32_t va = sbase + C::kVOff + s * C::kTile;
+        const uint64_t dv = s == 0 ? dv0 : dv1;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!mbar_wait(bar(hPFull + 2 * s + half), ph, abort_flag, args.dev_error)) return false;
@@ -368,9 +373,10 @@ __global__ void __launch_bounds__(kHThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const int ks = half * 4 + kk;
-            // V is MN-major here: 64-dim slabs kSlab apart, 8-key groups 1024 B apart.
-            mma_ts(tmem + kColO, tmem + (uint32_t)(128 * s + ks * 8),
-                   make_sdesc_sw128(va + (uint32_t)(ks * 2048), kSlab, 1024), id_pv, (p > 0 || ks > 0) ? 1u : 0u);
+            // V is MN-major here: 64-dim slabs kSlab apart, 8-key groups 1024 B
+            // apart, 16 keys (2048 B) per k-step.
+            mma_ts(tmem + kColO, tmem + (uint32_t)(128 * s + ks * 8), dv + (uint64_t)((ks * 2048) >> 4), id_pv,
+                   (p > 0 || ks > 0) ? 1u : 0u);
           }
         }
         tc_commit(bar(hVEmpty + s));

@@ -231,6 +231,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto s_col = [&](int h) -> uint32_t { return (uint32_t)(h * 128); };
       auto o_col = [&](int h) -> uint32_t { return (uint32_t)(NH * 128 + h * D); };
 
+      // Shared-memory matrix descriptors, built once (Q of each head, K and V of
+      // each stage); a k-step adds a compile-time offset (bytes >> 4).
+      const uint64_t dq0 = make_sdesc_sw128(sbase + C::kQOff, 16, 1024);
+      const uint64_t dq1 = make_sdesc_sw128(sbase + C::kQOff + C::kTileBytes, 16, 1024);
+      const uint64_t dk0 = make_sdesc_sw128(sbase + C::kKOff, 16, 1024);
+      const uint64_t dk1 = make_sdesc_sw128(sbase + C::kKOff + C::kKSlots * C::kTileBytes, 16, 1024);
+      const uint64_t dv0 = make_sdesc_sw128(sbase + C::kVOff, kChunkBytes, 1024);
+      const uint64_t dv1 = make_sdesc_sw128(sbase + C::kVOff + C::kTileBytes, kChunkBytes, 1024);
+      auto kstep_off = [](int ks) -> uint64_t {
+        return (uint64_t)(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
+      };
       auto issue_s = [&](int h, int p) -> bool {
         const int s = p % kStages;
         const uint32_t ph = (uint32_t)(p / kStages) & 1u;
@@ -239,16 +250,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(bar(kKFull + s), ph, abort_flag, args.dev_error)) return false;
           tc_fence_after();
         }
-        const uint32_t qa = sbase + C::kQOff + h * C::kTileBytes;
-        const uint32_t ka = sbase + C::kKOff + s * C::kKSlots * C::kTileBytes;
+        const uint64_t dq = h == 0 ? dq0 : dq1;
+        const uint64_t dk = s == 0 ? dk0 : dk1;
         const bool remote = pass_remote_ops<kKind>(sc, p);
         const uint32_t id_s = remote ? id_s_rem : id_s_loc;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (uint32_t)((ks >> 2) * kChunkBytes + (ks & 3) * 32);
-          mma_ss(tmem + s_col(h), make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-                 id_s, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ss(tmem + s_col(h), dq + kstep_off(ks), dk + kstep_off(ks), id_s, ks > 0 ? 1u : 0u);
         tc_commit(bar(kSFull + h));
         if (h == NH - 1) {
           tc_commit(bar(kKEmpty + s));
@@ -263,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = p % C::kVStages;
         const uint32_t ph = (uint32_t)(p / C::kVStages) & 1u;
         if (h == 0 && !mbar_wait(bar(kVFull + s), ph, abort_flag, args.dev_error)) return false;
-        const uint32_t va = sbase + C::kVOff + s * C::kTileBytes;
+        const uint64_t dv = s == 0 ? dv0 : dv1;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!mbar_wait(bar(kPFull + 2 * h + half), (uint32_t)p & 1u, abort_flag, args.dev_error)) return false;
@@ -274,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // V tile is MN-major for this product: 64-dim slabs kChunkBytes apart
             // (leading offset), 8-key groups 1024 B apart (stride offset).
             mma_ts(tmem + o_col(h), tmem + s_col(h) + (uint32_t)(ks * 8),
-                   make_sdesc_sw128(va + (uint32_t)(ks * 2048), kChunkBytes, 1024), id_pv,
+                   dv + (uint64_t)((ks * 2048) >> 4), id_pv,
                    (p > 0 || ks > 0) ? 1u : 0u);
           }
         }

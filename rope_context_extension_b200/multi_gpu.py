@@ -1,7 +1,9 @@
 """Multi-GPU layouts of the bifocal decode: one process per GPU.
 
 * Head sharding: each rank owns a contiguous group of KV heads (and their query
-  heads) and runs prefill / decode on it alone; no data crosses GPUs.
+  heads) and runs prefill / decode on it alone (head_shard_prefill /
+  head_shard_decode); no data crosses GPUs unless the caller asks for every
+  head's output in one place (one all-gather).
 * Sequence split: each rank holds a contiguous key range of every sequence's
   cache.  Positions, G and the band come from the global length, so the base
   keys never move; each rank computes its range's partial (O, LSE) with
@@ -29,6 +31,96 @@ def head_shard(Hkv: int, rank: int, world: int):
         raise ValueError("the KV heads must divide evenly over the ranks")
     n = Hkv // world
     return rank * n, n
+
+
+def head_shard_slices(Hq: int, Hkv: int, rank: int, world: int):
+    """(kv_begin, kv_count, q_begin, q_count) of `rank`: its KV heads and the query
+    heads that read them (query head h uses KV head h // (Hq / Hkv))."""
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    kb, kc = head_shard(Hkv, rank, world)
+    r = Hq // Hkv
+    return kb, kc, kb * r, kc * r
+
+
+def take_heads(x, begin: int, count: int, dim: int = 2):
+    """This rank's heads of a [..., heads, ...] tensor as a contiguous tensor of its own."""
+    return x.narrow(dim, begin, count).contiguous()
+
+
+def _gather_heads(x_r, head_dim: int, group):
+    """All-gather of per-rank head shards along `head_dim` (rank-major, so rank r's
+    heads land at [r * n, (r + 1) * n), matching head_shard)."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    parts = torch.empty((world,) + tuple(x_r.shape), dtype=x_r.dtype, device=x_r.device)
+    dist.all_gather_into_tensor(parts.view((world * x_r.shape[0],) + tuple(x_r.shape[1:])), x_r.contiguous(),
+                                group=group)
+    # [world, ..., n, ...] -> [..., world * n, ...]
+    moved = parts.movedim(0, head_dim)
+    shape = list(x_r.shape)
+    shape[head_dim] *= world
+    return moved.reshape(shape)
+
+
+def _default_prefill(q, k, v, kw):
+    import torch
+    from . import jetlong as jl
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device)
+    ws = kw.pop("workspace", None)
+    if ws is None:
+        ws = torch.empty(jl.jl_prefill_workspace_bytes(B, L, Hq, Hkv, D), dtype=torch.uint8, device=q.device)
+    jl.jl_bifocal_prefill(q, k, v, o, lse, workspace=ws, **kw)
+    return o, lse
+
+
+def _default_decode(q, kc, vc, kw):
+    import torch
+    from . import jetlong as jl
+    B, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    ws = kw.pop("workspace", None)
+    if ws is None:
+        ws = torch.zeros(jl.jl_decode_workspace_bytes(B, kw["L"], Hq, Hkv, D), dtype=torch.uint8, device=q.device)
+    jl.jl_bifocal_decode(q, kc, vc, o, lse, workspace=ws, **kw)
+    return o, lse
+
+
+def head_shard_prefill(q_r, k_r, v_r, *, group=None, gather: bool = False, prefill_fn=None, **kw):
+    """Bifocal prefill of this rank's KV-head group.
+
+    q_r [B, L, Hq / world, D], k_r / v_r [B, L, Hkv / world, D] hold the rank's
+    heads (take_heads of the full tensors, with the ranges of head_shard_slices);
+    the group is an independent problem with the same GQA ratio, G and band, so
+    the kernels run on it unchanged and nothing crosses GPUs.  Returns the rank's
+    (o [B, L, Hq / world, D], lse [B, Hq / world, L]); with gather=True the
+    all-ranks result (o [B, L, Hq, D], lse [B, Hq, L]) on every rank instead (one
+    all-gather each, only when the caller needs every head in one place).
+    Keyword arguments go to jl_bifocal_prefill (w0, w_pretrained, rope_base, ...).
+    """
+    import torch.distributed as dist
+    o_r, lse_r = (prefill_fn or _default_prefill)(q_r, k_r, v_r, dict(kw))
+    if not gather or not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return o_r, lse_r
+    return _gather_heads(o_r, 2, group), _gather_heads(lse_r, 1, group)
+
+
+def head_shard_decode(q_r, kc_r, vc_r, *, group=None, gather: bool = False, decode_fn=None, **kw):
+    """Bifocal decode of this rank's KV-head group: q_r [B, Hq / world, D], caches
+    [B, Lmax, Hkv / world, D].  Returns the rank's (o [B, Hq / world, D], lse
+    [B, Hq / world]) or, with gather=True, every head's on every rank.  Keyword
+    arguments go to jl_bifocal_decode (L, w0, w_pretrained, rope_base, ...)."""
+    import torch.distributed as dist
+    o_r, lse_r = (decode_fn or _default_decode)(q_r, kc_r, vc_r, dict(kw))
+    if not gather or not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return o_r, lse_r
+    return _gather_heads(o_r, 1, group), _gather_heads(lse_r, 1, group)
 
 
 def _default_partial(q, k_shard, v_shard, key_offset, key_count, total_len, kw):

@@ -1,7 +1,9 @@
-"""Sequence-split decode kernels on one GPU: each "rank" is one key range of
-the cache, run one after another (no rank waits on another), then the partial
-results are merged by jl_decode_combine.  The gather itself is covered over
-gloo in test_multigpu_cpu.py; this file pins the kernels.
+"""Multi-GPU layouts' kernels on one GPU, each "rank" run one after another (no
+rank waits on another).  Sequence split: each rank is one key range of the
+cache, and the partial results are merged by jl_decode_combine.  Head sharding:
+each rank is one KV-head group with its query heads, as contiguous tensors of
+its own.  The gathers themselves are covered over gloo in test_multigpu_cpu.py;
+this file pins the kernels.
 """
 
 import numpy as np
@@ -72,3 +74,47 @@ def test_sequence_split_driver_single_rank_equals_decode():
     p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=base)
     o_ref, l_ref = jo.decode(q.double().numpy(), kc.double().numpy(), vc.double().numpy(), p)
     assert_close(o.float().cpu().numpy(), o_ref, lse.cpu().numpy(), l_ref, "driver, one rank")
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_shard_groups_equal_the_whole_problem(world):
+    # Prefill and decode per KV-head group (the kernels see a smaller problem
+    # with the same GQA ratio, G and band); concatenated over the groups they
+    # equal one call on every head (prefill bit for bit: each head's result
+    # does not depend on the others; decode within rounding, since the split
+    # count follows the number of (sequence, KV head) pairs) and the oracle.
+    B, L, Hq, Hkv, D, W, w0 = 1, 2000, 16, 4, 128, 600, 300
+    q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=19, outlier_frac=0.01)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    kw = dict(w0=w0, w_pretrained=W, rope_base=1e6)
+    o_all, l_all = multi_gpu.head_shard_prefill(qd, kd, vd, **kw)
+    q1 = qd[:, L - 1].contiguous()
+    od_all, ld_all = multi_gpu.head_shard_decode(q1, kd, vd, L=L, **kw)
+    os_, ls_, ods, lds = [], [], [], []
+    for rank in range(world):
+        kb, kc_, qb, qc_ = multi_gpu.head_shard_slices(Hq, Hkv, rank, world)
+        q_r = multi_gpu.take_heads(qd, qb, qc_)
+        k_r, v_r = multi_gpu.take_heads(kd, kb, kc_), multi_gpu.take_heads(vd, kb, kc_)
+        o_r, l_r = multi_gpu.head_shard_prefill(q_r, k_r, v_r, **kw)
+        od_r, ld_r = multi_gpu.head_shard_decode(multi_gpu.take_heads(q1, qb, qc_, dim=1), k_r, v_r, L=L, **kw)
+        os_.append(o_r)
+        ls_.append(l_r)
+        ods.append(od_r)
+        lds.append(ld_r)
+    torch.cuda.synchronize()
+    o_sh, l_sh = torch.cat(os_, dim=2), torch.cat(ls_, dim=1)
+    od_sh, ld_sh = torch.cat(ods, dim=1), torch.cat(lds, dim=1)
+    assert torch.equal(o_sh, o_all) and torch.equal(l_sh, l_all)
+    assert (od_sh.float() - od_all.float()).abs().max().item() <= 2e-2
+    assert (ld_sh - ld_all).abs().max().item() <= 1e-3
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=1e6)
+    rows = np.array([0, 299, 300, 301, 1023, 1024, 1999])
+    ref = {}
+    for h in (0, 5, 15):
+        g = h // (Hq // Hkv)
+        ref[h] = jo.attention_rows(q[0, rows, h].double().numpy(), rows, k[0, :, g].double().numpy(),
+                                   v[0, :, g].double().numpy(), p)
+        assert_close(o_sh[0, rows, h].float().cpu().numpy(), ref[h][0], l_sh[0, h, rows].cpu().numpy(), ref[h][1],
+                     f"head shard h{h}")
+    od_ref, ld_ref = jo.decode(q[:, L - 1].float().numpy(), k.float().numpy(), v.float().numpy(), p)
+    assert_close(od_sh.float().cpu().numpy(), od_ref, ld_sh.cpu().numpy(), ld_ref, "head shard decode")
