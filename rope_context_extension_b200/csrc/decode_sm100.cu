@@ -221,17 +221,17 @@ __global__ void __maxnreg__(JL_DEC_MAXNREG)
     const int q64 = kDecKeys / G;
     for (int idx = threadIdx.x; idx < (18 + kDecWarps) * H2; idx += kCons) {
       const int row = idx / H2, t = idx % H2;
-      double turns;
+      int64_t turns;  // the angle in units of theta_t (an integer)
       if (row < 16) {
-        turns = -(double)row;
+        turns = -row;
       } else if (row < 18) {
-        turns = -(double)(q64 + (row - 16) - kDecKeys);  // -(dk(j0 + kDecKeys) - dk(j0))
+        turns = -(q64 + (row - 16) - kDecKeys);  // -(dk(j0 + kDecKeys) - dk(j0))
       } else {
         const int64_t j0 = (int64_t)t_begin * kDecKeys + 16 * (row - 18) + key_off;  // position
-        turns = (double)(dq - (j0 / G - j0));
+        turns = dq - (j0 / G - j0);
       }
       double sn, cs;
-      sincos(turns * args.theta[t], &sn, &cs);
+      sincos_int_angle(turns, args.u_hi[t], args.u_lo[t], &sn, &cs);
       // E and F rows hold (c_t, c_t+1, s_t, s_t+1) for even t; Q0 rows (c_t, s_t)
       float* dst = row < 16 ? reinterpret_cast<float*>(E) + row * (C::kERow / 4)
                             : reinterpret_cast<float*>(F) + (row - 16) * D;

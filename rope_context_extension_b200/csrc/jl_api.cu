@@ -67,6 +67,18 @@ void fill_theta(double* theta, int D, double base) {
   for (int t = 0; t < D / 2; ++t) theta[t] = std::pow(base, -2.0 * t / D);
 }
 
+// theta_t / (2 pi) as u_hi + u_lo, u_hi rounded to 22 significant bits (so that
+// n * u_hi is exact in fp64 for |n| < 2^31; see sincos_int_angle).
+void fill_turns(double* u_hi, double* u_lo, const double* theta, int D) {
+  for (int t = 0; t < D / 2; ++t) {
+    const double u = theta[t] / 6.283185307179586;
+    int e = 0;
+    const double m = std::frexp(u, &e);
+    u_hi[t] = std::ldexp(std::nearbyint(std::ldexp(m, 22)), e - 22);
+    u_lo[t] = u - u_hi[t];
+  }
+}
+
 constexpr int kMaxGridYZ = 65535;  // CUDA's limit on a grid's y and z dimensions
 
 int common_checks(int B, int L, int Hq, int Hkv, int D, int w0, int w_pretrained, double rope_base, int mode) {
@@ -293,6 +305,7 @@ int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double
   RotateArgs ra;
   std::memset(&ra, 0, sizeof(ra));
   fill_theta(ra.theta, pp.D, rope_base);
+  fill_turns(ra.u_hi, ra.u_lo, ra.theta, pp.D);
   ra.G = G;
   ra.shift = jl::query_shift(w0, G, mode & JL_QSHIFT_SELF_EXTEND);
   ra.B = pp.B;
@@ -335,6 +348,7 @@ int correction_launch(const PrefillProblem& pp, int w0, int w_pretrained, double
 // R(-theta_t 16 a) for a < 8, formed in fp64 and rounded to fp32.
 void fill_hilo_tables(jl::PrefillHiloArgs& a, int D, double rope_base) {
   fill_theta(a.theta, D, rope_base);
+  fill_turns(a.u_hi, a.u_lo, a.theta, D);
   for (int t = 0; t < D / 2; ++t) {
     for (int b = 0; b < 16; ++b)
       a.t1[t * 16 + b] = make_float2((float)std::cos(b * a.theta[t]), (float)-std::sin(b * a.theta[t]));
@@ -634,6 +648,7 @@ int decode_launch(const void* q, const void* k_cache, const void* v_cache, int64
   a.qshift = mode & JL_QSHIFT_SELF_EXTEND;
   a.scale_log2 = resolve_scale(softmax_scale, D) * 1.4426950408889634f;
   fill_theta(a.theta, D, rope_base);
+  fill_turns(a.u_hi, a.u_lo, a.theta, D);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (compact && cudaMemsetAsync(a.counters, 0, (size_t)B * Hkv * sizeof(int), s) != cudaSuccess)
     return JL_ERR_CUDA;
@@ -739,6 +754,7 @@ int jl_rope_append(const void* q_raw, const void* k_raw, const void* v_new, cons
   a.Hkv = Hkv;
   a.dev_error = dev_error;
   fill_theta(a.theta, head_dim, rope_base);
+  fill_turns(a.u_hi, a.u_lo, a.theta, head_dim);
   if (jl::launch_rope_append(a, head_dim, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }

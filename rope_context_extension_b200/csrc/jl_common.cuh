@@ -232,6 +232,19 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// cos and sin of the angle n * theta for an integer n (|n| < 2^31), given
+// theta / (2 pi) = u_hi + u_lo with u_hi holding at most 22 significant bits
+// (fill_turns on the host).  n * u_hi is then exact, so the whole turns are
+// removed exactly and sincos only ever sees an angle in [-pi, pi] (its fast
+// path), whatever the size of n * theta.
+__device__ __forceinline__ void sincos_int_angle(int64_t n, double u_hi, double u_lo, double* s, double* c) {
+  double a = (double)n * u_hi;  // exact
+  a -= rint(a);
+  double f = a + (double)n * u_lo;
+  f -= rint(f);
+  sincos(f * 6.283185307179586, s, c);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -21,6 +21,7 @@ struct RotateArgs {
   int64_t G, shift;  // group size and query shift
   int* dev_error;    // device int or null: set to kDevRange when a rotated value leaves fp16's range
   double theta[kMaxHalfDim];
+  double u_hi[kMaxHalfDim], u_lo[kMaxHalfDim];  // theta_t / (2 pi), split for exact turn removal
 };
 cudaError_t launch_rotate_rows(const RotateArgs& args, int D, cudaStream_t stream);
 
@@ -65,6 +66,7 @@ struct PrefillHiloArgs {
   int64_t G, shift;        // group size and query shift (from the total length q_off + Lq)
   float scale_log2;        // softmax scale * log2(e)
   double theta[kMaxHalfDim];
+  double u_hi[kMaxHalfDim], u_lo[kMaxHalfDim];  // theta_t / (2 pi), split for exact turn removal
   float2 t1[kMaxHalfDim * 16];   // R(-theta_t b) for b < 16, [t][b] (cos, sin)
   float2 t16[kMaxHalfDim * 8];   // R(-theta_t 16 a) for a < 8, [t][a]
 };
@@ -90,6 +92,7 @@ struct DecodeArgs {
   int w0, w_pretrained, qshift;
   float scale_log2;
   double theta[kMaxHalfDim];
+  double u_hi[kMaxHalfDim], u_lo[kMaxHalfDim];  // theta_t / (2 pi), split for exact turn removal
 };
 // dev_error value for a sequence length outside [1, cache_len] (varlen decode)
 constexpr int kDevBadLength = 2;
@@ -145,6 +148,7 @@ struct AppendArgs {
   int B, Hq, Hkv;
   int* dev_error;
   double theta[kMaxHalfDim];
+  double u_hi[kMaxHalfDim], u_lo[kMaxHalfDim];  // theta_t / (2 pi), split for exact turn removal
 };
 cudaError_t launch_rope_append(const AppendArgs& a, int D, cudaStream_t stream);
 

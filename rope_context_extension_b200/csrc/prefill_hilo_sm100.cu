@@ -25,9 +25,9 @@
 //     instead of 2^-11 for one fp16 product (which is what a key of large norm
 //     that dominates a softmax row turns into an LSE error).
 // In-kernel correction angles theta_t * d come from a factor R(theta_t (d_x0 -
-// 16 a)) for the row set's first row x0 (fp64: one sincos per CTA, then an
-// fp64 recurrence from one key tile to the next) times a table R(-theta_t b),
-// with d = d_x0 - (16 a + b) inside the set.
+// 16 a)) for the row set's first row x0 (fp64: one sincos per CTA, its whole
+// turns removed exactly first, then an fp64 recurrence from one key tile to the
+// next) times a table R(-theta_t b), with d = d_x0 - (16 a + b) inside the set.
 //
 // Each 128 x 128 (query block, key block) tile is visited once per score set it
 // needs (remote passes first, then local passes; a tile straddling the band
@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
       const int t = e / TPT;
       const int a0 = (e % TPT) * APT;
       double sn, cs;
-      sincos(args.theta[t] * (double)base, &sn, &cs);
+      sincos_int_angle(base, args.u_hi[t], args.u_lo[t], &sn, &cs);
       const float cb = (float)cs, sb = (float)sn;
 #pragma unroll
       for (int j = 0; j < APT; ++j) {
@@ -709,11 +709,11 @@ __global__ void __launch_bounds__(kHThreads, 1)
       constexpr int APT = 8 / TPT;
       const int ft = e / TPT;
       const int fa0 = (e % TPT) * APT;
-      const double th = args.theta[ft];
+      const double uh = args.u_hi[ft], ul = args.u_lo[ft];
       const int64_t s_lo = 128 - (128 + G - 1) / G;
       double st_s[2], st_c[2];
-      sincos(th * (double)s_lo, &st_s[0], &st_c[0]);
-      sincos(th * (double)(s_lo + 1), &st_s[1], &st_c[1]);
+      sincos_int_angle(s_lo, uh, ul, &st_s[0], &st_c[0]);
+      sincos_int_angle(s_lo + 1, uh, ul, &st_s[1], &st_c[1]);
       double kb_c = 1.0, kb_s = 0.0;
       int64_t prev_dk0 = 0;
       bool have_base = false;
@@ -723,7 +723,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
           const int64_t j0 = (int64_t)ps.nb * 128;
           const int64_t dk0 = j0 / G - j0;
           if (!have_base) {
-            sincos(th * (double)dk0, &kb_s, &kb_c);
+            sincos_int_angle(dk0, uh, ul, &kb_s, &kb_c);
             have_base = true;
           } else {
             const int i = (int)(dk0 - prev_dk0 - s_lo);  // 0 or 1

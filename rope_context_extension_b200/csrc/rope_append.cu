@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(128) rope_append_kernel(const __grid_constant_
   }
   for (int t = threadIdx.x; t < H2; t += blockDim.x) {
     double s, c;
-    sincos((double)p * a.theta[t], &s, &c);
+    sincos_int_angle(p, a.u_hi[t], a.u_lo[t], &s, &c);
     cs[t] = make_float2((float)c, (float)s);
   }
   __syncthreads();

@@ -9,7 +9,8 @@
 // caller-owned scratch; the input tensors (the KV cache) are never touched.
 //
 // Angles reach ~1e5 rad at 128K tokens, so they are formed and reduced in fp64
-// (one sincos per (row, pair), shared by every head of the row); the rotation
+// (one sincos per (row, pair), shared by every head of the row, with the whole
+// turns removed exactly first: sincos_int_angle); the rotation
 // itself is fp32 and the output is rounded to fp16 (round-to-nearest-even),
 // optionally with the rounding residual as a second fp16 row (hi + lo carry
 // about 22 significant bits): the rotated rows only feed the score products,
@@ -42,9 +43,8 @@ __global__ void __launch_bounds__(kRotThreads)
     if (i < args.row_end) {
       const int64_t pos = i + args.pos_off;
       const int64_t target = args.is_query ? query_remote(pos, args.G, args.shift) : key_remote(pos, args.G);
-      const double ang = (double)(target - pos) * args.theta[t];
       double s, c;
-      sincos(ang, &s, &c);
+      sincos_int_angle(target - pos, args.u_hi[t], args.u_lo[t], &s, &c);
       v = make_float2((float)c, (float)s);
     }
     cs[r][t] = v;
