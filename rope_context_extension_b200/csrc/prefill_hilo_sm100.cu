@@ -51,9 +51,19 @@ namespace {
 constexpr int kHThreads = 384;
 constexpr int kHStages = 2;
 constexpr int kHLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
-constexpr int kHLowRegs = 104;     // warpgroup 0: TMA producer, MMA issuer
-constexpr int kHHighRegs = 200;    // warpgroups 1-2: softmax, rotation
-static_assert(128 * kHLowRegs + 256 * kHHighRegs <= kHThreads * kHLaunchRegs, "register split exceeds the launch pool");
+// Registers per thread of each warpgroup after setmaxnreg.  With key tiles
+// rotated in the kernel the rotation warpgroup holds two key rows in flight
+// and needs as many as the softmax; otherwise it only sets up the query
+// operands, and the producer / MMA warpgroup gets the difference (the MMA
+// thread's loop then keeps all its state in registers).
+template <bool kRotK>
+struct HRegs {
+  static constexpr int kProducer = kRotK ? 104 : 152;  // warpgroup 0: TMA producer, MMA issuer
+  static constexpr int kSoftmax = 200;                 // warpgroup 1
+  static constexpr int kRotation = kRotK ? 200 : 152;  // warpgroup 2
+  static_assert(128 * (kProducer + kSoftmax + kRotation) <= kHThreads * kHLaunchRegs,
+                "register split exceeds the launch pool");
+};
 constexpr int kSlab = 128 * 128;  // one 128-row x 128-byte swizzled slab
 
 template <int D>
@@ -74,20 +84,24 @@ struct HCfg {
 };
 
 // barrier slots
+// Every barrier the MMA thread commits to or waits on costs tensor-pipe time
+// (the issuing thread has no slack between products), so each signal serves
+// every consumer that can use it: the score commit of a pass also frees the
+// key stage it read, and the P V commit also tells the softmax that O holds
+// that pass's product.  Stage s, S buffer s and V stage s all belong to the
+// passes p with p % 2 == s.
 enum {
   hKFull = 0,         // [stage]: rotated (or copied) key tile in shared memory
-  hKEmpty = 2,        // [stage]: the score products reading it have completed
-  hVFull = 4,
-  hVEmpty = 6,
-  hSFull = 8,         // [S buffer]
-  hPFull = 10,        // [S buffer][64-key half of P]
-  hPVDone = 14,       // O += P V of the latest pass has completed
-  hQReady = 16,       // the query operands are in TMEM (phase 0: first pass kind, 1: after the switch)
-  hQEmpty = 17,       // the last product reading the first query operands has completed
-  hCReady = 18,       // rotation warpgroup: factor table of the next tile written
-  hOFinal = 19,
-  hDrain = 20,
-  hNumBars = 21
+  hVFull = 2,         // [stage]
+  hVEmpty = 4,        // [stage]: O += P V of the stage's latest pass has completed
+  hSFull = 6,         // [S buffer]: scores complete; the key stage they read is free
+  hPFull = 8,         // [S buffer]: P written over S
+  hQReady = 10,       // the query operands are in TMEM (phase 0: first pass kind, 1: after the switch)
+  hQEmpty = 11,       // the last product reading the first query operands has completed
+  hCReady = 12,       // rotation warpgroup: factor table of the next tile written
+  hOFinal = 13,
+  hDrain = 14,
+  hNumBars = 15
 };
 static_assert(hNumBars * 8 <= 192, "barrier block overflow");
 
@@ -238,14 +252,11 @@ __global__ void __launch_bounds__(kHThreads, 1)
     *abort_flag = 0;
     for (int s = 0; s < kHStages; ++s) {
       mbar_init(bar(hKFull + s), kRotK ? 128 : 1);
-      mbar_init(bar(hKEmpty + s), 1);
       mbar_init(bar(hVFull + s), 1);
       mbar_init(bar(hVEmpty + s), 1);
       mbar_init(bar(hSFull + s), 1);
-      mbar_init(bar(hPFull + 2 * s), 128);
-      mbar_init(bar(hPFull + 2 * s + 1), 128);
+      mbar_init(bar(hPFull + s), 128);
     }
-    mbar_init(bar(hPVDone), 1);
     mbar_init(bar(hQReady), 128);
     mbar_init(bar(hQEmpty), 1);
     mbar_init(bar(hCReady), 128);
@@ -270,7 +281,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
   const int p_switch = sc.n_rem;  // first local pass (fused method)
 
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHLowRegs));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(HRegs<kRotK>::kProducer));
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ producer
       tma_prefetch_map(&tm_v);
@@ -286,7 +297,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
         const uint32_t ph = (uint32_t)(p >> 1) & 1u;
         const HPass ps = hilo_pass<kKind>(sc, p);
         if (!kRotK) {
-          if (!(ok = mbar_wait(bar(hKEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
+          if (!(ok = mbar_wait(bar(hSFull + s), ph ^ 1u, abort_flag, args.dev_error))) break;
           const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
           mbar_arrive_expect_tx(bar(hKFull + s), (uint32_t)((ps.remote ? 2 : 1) * C::kTile));
           for (int c = 0; c < C::kChunks; ++c) {
@@ -327,6 +338,9 @@ __global__ void __launch_bounds__(kHThreads, 1)
       const uint64_t dv0 = make_sdesc_sw128(sbase + C::kVOff, kSlab, 1024);
       const uint64_t dv1 = make_sdesc_sw128(sbase + C::kVOff + C::kTile, kSlab, 1024);
       auto kstep_off = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * kSlab + (ks & 3) * 32) >> 4); };
+      // passes with corrected (hi + lo) operands: the fused method's remote
+      // passes come first; the single-kind calls use one operand kind
+      const int n_hilo = kKind == kBifocal ? sc.n_rem : (kKind != kWindowBase ? npass : 0);
       auto issue_s = [&](int p) -> bool {
         const int s = p & 1;
         const uint32_t ph = (uint32_t)(p >> 1) & 1u;
@@ -335,52 +349,47 @@ __global__ void __launch_bounds__(kHThreads, 1)
         }
         if (!mbar_wait(bar(hKFull + s), ph, abort_flag, args.dev_error)) return false;
         tc_fence_after();
-        const HPass ps = hilo_pass<kKind>(sc, p);
         const uint32_t d = tmem + (uint32_t)(128 * s);
         // descriptors of the stage's K_hi / K_lo tiles (k-step offsets are
         // added below as compile-time constants: one add per MMA)
         const uint64_t dkh = s == 0 ? dk_hi0 : dk_hi1;
-        const uint64_t dkl = dkh + (uint64_t)(C::kTile >> 4);
-        const uint32_t id_s = ps.remote ? id_rem : id_loc;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_s, ks > 0 ? 1u : 0u);
-        if (ps.remote) {
-          // + Q_hi K_lo + Q_lo K_hi into the same accumulator
+        if (p < n_hilo) {
+          const uint64_t dkl = dkh + (uint64_t)(C::kTile >> 4);
+          // Q_hi K_hi + Q_hi K_lo + Q_lo K_hi into one accumulator
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkl + kstep_off(ks), id_s, 1u);
+            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_rem, ks > 0 ? 1u : 0u);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(d, tmem + kColQB + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_s, 1u);
+            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkl + kstep_off(ks), id_rem, 1u);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ts(d, tmem + kColQB + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_rem, 1u);
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_loc, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(hSFull + s));
-        tc_commit(bar(hKEmpty + s));
         if (q_switch && p == p_switch - 1) tc_commit(bar(hQEmpty));
         return true;
       };
-      // O += P V in two 64-key halves, each issued as soon as the softmax has
-      // written that half of P.
+      // O += P V once the softmax has written all of P.
       auto issue_pv = [&](int p) -> bool {
         const int s = p & 1;
         const uint32_t ph = (uint32_t)(p >> 1) & 1u;
         if (!mbar_wait(bar(hVFull + s), ph, abort_flag, args.dev_error)) return false;
+        if (!mbar_wait(bar(hPFull + s), ph, abort_flag, args.dev_error)) return false;
+        tc_fence_after();
         const uint64_t dv = s == 0 ? dv0 : dv1;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if (!mbar_wait(bar(hPFull + 2 * s + half), ph, abort_flag, args.dev_error)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int ks = half * 4 + kk;
-            // V is MN-major here: 64-dim slabs kSlab apart, 8-key groups 1024 B
-            // apart, 16 keys (2048 B) per k-step.
-            mma_ts(tmem + kColO, tmem + (uint32_t)(128 * s + ks * 8), dv + (uint64_t)((ks * 2048) >> 4), id_pv,
-                   (p > 0 || ks > 0) ? 1u : 0u);
-          }
+        for (int ks = 0; ks < 8; ++ks) {
+          // V is MN-major here: 64-dim slabs kSlab apart, 8-key groups 1024 B
+          // apart, 16 keys (2048 B) per k-step.
+          mma_ts(tmem + kColO, tmem + (uint32_t)(128 * s + ks * 8), dv + (uint64_t)((ks * 2048) >> 4), id_pv,
+                 (p > 0 || ks > 0) ? 1u : 0u);
         }
         tc_commit(bar(hVEmpty + s));
-        tc_commit(bar(hPVDone));
         return true;
       };
       bool ok = true;
@@ -402,7 +411,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
       }
     }
   } else if (warp < 8) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHHighRegs));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(HRegs<kRotK>::kSoftmax));
     // ------------------------------------------------------------ softmax
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
@@ -490,8 +499,8 @@ __global__ void __launch_bounds__(kHThreads, 1)
         m_used = m_new;
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-      // O must be rescaled before this pass's P V; in the (rare) passes that
-      // need it, both halves of P are released after the rescale.
+      // O must be rescaled before this pass's P V: in the (rare) passes that
+      // need it, P is released after the rescale.
       const bool resc = __any_sync(0xffffffffu, rescale_o) && p > 0;
       const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-msub, -msub);
       uint64_t acc[2] = {0ull, 0ull};
@@ -512,18 +521,12 @@ __global__ void __launch_bounds__(kHThreads, 1)
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) pk[k] = pair_exp(1, k);
-        if (!resc) {
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(bar(hPFull + 2 * s));
-        }
-#pragma unroll
-        for (int k = 8; k < 32; ++k) pk[k] = pair_exp(1, k);
+        for (int k = 0; k < 32; ++k) pk[k] = pair_exp(1, k);
         tmem_st32(s_addr + 32, pk);
         if (resc) {
           // O must hold the previous pass's product first.
-          bool okw = mbar_wait(bar(hPVDone), (uint32_t)(p - 1) & 1u, abort_flag, args.dev_error);
+          bool okw = mbar_wait(bar(hVEmpty + ((p - 1) & 1)), (uint32_t)((p - 1) >> 1) & 1u, abort_flag,
+                               args.dev_error);
           okw = __all_sync(0xffffffffu, okw);
           if (!okw) {
             ok = false;
@@ -542,8 +545,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        if (resc) mbar_arrive(bar(hPFull + 2 * s));
-        mbar_arrive(bar(hPFull + 2 * s + 1));
+        mbar_arrive(bar(hPFull + s));
       }
       {
         float a0, a1;
@@ -598,7 +600,10 @@ __global__ void __launch_bounds__(kHThreads, 1)
       }
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHHighRegs));
+    if constexpr (kRotK)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(HRegs<kRotK>::kRotation));
+    else
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(HRegs<kRotK>::kRotation));
     // ------------------------------------------------------------ rotation
     const int wq = warp & 3;
     const int e = wq * 32 + lane;  // query row of the block / key row of the tile
@@ -753,7 +758,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
         const HPass ps = hilo_pass<kKind>(sc, p);
         // every thread's factors for tile p, then the stage's previous reader
         if (!mbar_wait(bar(hCReady), (uint32_t)(p + 1) & 1u, abort_flag, args.dev_error)) return false;
-        if (!mbar_wait(bar(hKEmpty + s), ((uint32_t)(p >> 1) & 1u) ^ 1u, abort_flag, args.dev_error)) return false;
+        if (!mbar_wait(bar(hSFull + s), ((uint32_t)(p >> 1) & 1u) ^ 1u, abort_flag, args.dev_error)) return false;
         const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
         if (ps.remote) {
           const int64_t j0 = (int64_t)ps.nb * 128;
