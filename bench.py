@@ -106,59 +106,122 @@ def sources_hash(files):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """SM clock, power and clock-event (throttle) reasons sampled every 20 ms
+    through NVML while the timed region runs (nvidia-smi at 200 ms when NVML
+    is not importable).  Only samples taken between mark_begin() and
+    mark_end() count, so the median is the clock under load."""
 
+    # NVML clock-event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device: int):
+        self.dev = torch_device
+        self.samples = []  # (time, sm_mhz, power_w, reasons)
+        self.window = [None, None]
+        self.stop_evt = threading.Event()
         self.thread = None
+        self.proc = None
+        self.nvml = None
+        self.handle = None
+        self.smax = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        self.nvml = pynvml
+        uuid = str(getattr(torch.cuda.get_device_properties(self.dev), "uuid", "") or "")
+        if uuid:
+            try:
+                return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        idx = int(vis.split(",")[self.dev]) if vis and vis.split(",")[0].isdigit() else self.dev
+        return pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+            self.handle = self._nvml_handle()
+            nv = self.nvml
+            self.smax = float(nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self.stop_evt.is_set():
+                    t = time.perf_counter()
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1e3
+                        rs = int(get_reasons(self.handle))
+                    except Exception:
+                        break
+                    self.samples.append((t, sm, pw, rs))
+                    self.stop_evt.wait(0.02)
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.handle = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        if self.thread:
-            self.thread.join(timeout=2)
-        sm, smax, reasons = [], None, set()
+    def _read_smi(self):
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.strip().split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                sm, self.smax = float(parts[1]), float(parts[2])
+                pw = float(parts[3])
             except ValueError:
                 continue
+            rs = 0
             for n, val in zip(names, parts[5:9]):
                 if val.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                    rs |= self.REASONS[n]
+            self.samples.append((time.perf_counter(), sm, pw, rs))
+
+    def mark_begin(self):
+        self.window[0] = time.perf_counter()
+
+    def mark_end(self):
+        self.window[1] = time.perf_counter()
+
+    def stop(self):
+        self.stop_evt.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        if self.handle is None and self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no NVML and no nvidia-smi"]}
+        t0 = self.window[0] if self.window[0] is not None else -math.inf
+        t1 = self.window[1] if self.window[1] is not None else math.inf
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        reasons = sorted(n for n, bit in self.REASONS.items() if any(x[3] & bit for x in inside))
+        return {"sm_mhz": statistics.median(x[1] for x in inside) if inside else None, "sm_max_mhz": self.smax,
+                "sm_mhz_min": min(x[1] for x in inside) if inside else None,
+                "power_w_median": round(statistics.median(x[2] for x in inside), 1) if inside else None,
+                "reasons": reasons, "samples": len(inside),
+                "source": "nvml 20 ms" if self.handle is not None else "nvidia-smi 200 ms"}
 
 
 def dist_setup(n_gpus):
@@ -320,12 +383,14 @@ def run_ours(args):
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
+    clocks.mark_begin()
     t0.record(stream)
     for i in range(K):
         prefill_step(pev[i])
         decode_step(dev_[i])
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     barrier(world)
     clk = clocks.stop()
     if int(err.item()) != 0:
@@ -378,11 +443,13 @@ def run_ours(args):
         a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
+        sampler.mark_begin()
         a_.record(stream)
         for _ in range(reps):
             call()
         b_.record(stream)
         torch.cuda.synchronize()
+        sampler.mark_end()
         barrier(world)
         clk_ = sampler.stop()
         ms = max_over_ranks(a_.elapsed_time(b_) / reps, world)
@@ -627,6 +694,10 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": tensor_peak,
                          "unit": "TFLOP/s", "frac": round(attn_tflops / tensor_peak, 4),
                          "traffic": traffic.get("prefill_attention", {}).get("bytes_per_launch"),
+                         "traffic_smaller_sizes": traffic.get("prefill_attention", {}).get("measured_smaller"),
+                         "traffic_note": "DRAM bytes per launch measured by ncu at the profiling sizes (same G and "
+                                         "w0 / L); they do not grow in proportion to L, so the 128K launch's "
+                                         "traffic is not extrapolated",
                          "kernel": "bifocal_prefill_hilo_kernel<128, false, 0>",
                          "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a multi-second loop)",
                          "executed_tflops": round(exec_flop / (attn_ms_max * 1e-3) / 1e12, 2),
@@ -634,8 +705,14 @@ def run_ours(args):
                          "executed_note": "tensor-core flop actually issued: three score products per remote tile "
                                           "(hi + lo), one per local tile, one P V per tile",
                          "per_ghz": {"kernel_tflops_per_sm_ghz": round(attn_tflops / sm_ghz, 1) if sm_ghz else None,
+                                     "kernel_executed_tflops_per_sm_ghz":
+                                         round(exec_flop / (attn_ms_max * 1e-3) / 1e12 / sm_ghz, 1) if sm_ghz else None,
                                      "peak_tflops_per_sm_ghz": round(tensor_peak / peak_ghz, 1) if peak_ghz else None,
-                                     "note": "TFLOP/s divided by the median SM clock sampled while each ran"}},
+                                     "tensor_core_tflops_per_sm_ghz": round(8192 * 148 / 1e3, 1),
+                                     "note": "TFLOP/s divided by the median SM clock sampled while each ran "
+                                             "(the step's clocks for the kernel, the peak file's for cuBLAS); "
+                                             "the tensor-core figure is 8192 flop per clock per SM (one "
+                                             "128 x 128 x 16 product per 64 clocks, measured) x 148 SMs"}},
             "e2e": e2e,
             "gpu_launches": K * 3,
             "gpu_launches_decode_loops": dloop8["reps"] + dloop1["reps"],
