@@ -90,12 +90,25 @@ struct HCfg {
 // key stage it read, and the P V commit also tells the softmax that O holds
 // that pass's product.  Stage s, S buffer s and V stage s all belong to the
 // passes p with p % 2 == s.
+//
+// With pre-rotated keys (the default) the MMA thread waits once per pass:
+// hReady[s] gathers everything pass p (p % 2 == s) needs before its P V and
+// the next score products of the same parity.  Phase 0 of hReady[s] holds
+// K(s) and V(s) for the first two passes (the softmax arrives once at the
+// start); phase n >= 1 is pass p = 2 (n - 1) + s: P(p) written (128 softmax
+// arrivals), V(p) and K(p + 2) landed (the producer's arrival comes with
+// K(p + 2), or alone when there is none).  Each party registers on phase n
+// only after something it waited for shows phase n - 1 complete: the
+// producer's K(p + 2) follows S(p), V(p)'s bytes follow P V of pass p - 2,
+// and P(p) follows S(p), all issued after the MMA thread's wait on phase n - 1.
+// With keys corrected in the kernel, hReady[s] is "key tile p in shared
+// memory" (128 rotation-thread arrivals) and V and P have barriers of their own.
 enum {
-  hKFull = 0,         // [stage]: rotated (or copied) key tile in shared memory
-  hVFull = 2,         // [stage]
+  hReady = 0,         // [parity]: the pass barrier above (key tile p with in-kernel keys)
+  hVFull = 2,         // [stage] (in-kernel keys only)
   hVEmpty = 4,        // [stage]: O += P V of the stage's latest pass has completed
   hSFull = 6,         // [S buffer]: scores complete; the key stage they read is free
-  hPFull = 8,         // [S buffer]: P written over S
+  hPFull = 8,         // [S buffer]: P written over S (in-kernel keys only)
   hQReady = 10,       // the query operands are in TMEM (phase 0: first pass kind, 1: after the switch)
   hQEmpty = 11,       // the last product reading the first query operands has completed
   hCReady = 12,       // rotation warpgroup: factor table of the next tile written
@@ -251,7 +264,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int s = 0; s < kHStages; ++s) {
-      mbar_init(bar(hKFull + s), kRotK ? 128 : 1);
+      mbar_init(bar(hReady + s), kRotK ? 128 : 129);
       mbar_init(bar(hVFull + s), 1);
       mbar_init(bar(hVEmpty + s), 1);
       mbar_init(bar(hSFull + s), 1);
@@ -296,33 +309,57 @@ __global__ void __launch_bounds__(kHThreads, 1)
         const int s = p & 1;
         const uint32_t ph = (uint32_t)(p >> 1) & 1u;
         const HPass ps = hilo_pass<kKind>(sc, p);
-        if (!kRotK) {
+        const uint32_t vdst = sbase + C::kVOff + s * C::kTile;
+        if constexpr (!kRotK) {
+          // K(p): its stage is free once S(p - 2) has completed; it belongs to
+          // the phase of pass p - 2 (phase 0 for p < 2, together with V(p))
           if (!(ok = mbar_wait(bar(hSFull + s), ph ^ 1u, abort_flag, args.dev_error))) break;
           const uint32_t khi = sbase + C::kKOff + s * 2 * C::kTile;
-          mbar_arrive_expect_tx(bar(hKFull + s), (uint32_t)((ps.remote ? 2 : 1) * C::kTile));
+          const uint32_t kbytes = (uint32_t)((ps.remote ? 2 : 1) * C::kTile);
+          mbar_arrive_expect_tx(bar(hReady + s), p < 2 ? kbytes + (uint32_t)C::kTile : kbytes);
           for (int c = 0; c < C::kChunks; ++c) {
             if (ps.remote) {
-              tma_load_4d(khi + c * kSlab, &tm_kh, bar(hKFull + s), c * 64, kvh, ps.nb * 128, b);
-              tma_load_4d(khi + C::kTile + c * kSlab, &tm_kl, bar(hKFull + s), c * 64, kvh, ps.nb * 128, b);
+              tma_load_4d(khi + c * kSlab, &tm_kh, bar(hReady + s), c * 64, kvh, ps.nb * 128, b);
+              tma_load_4d(khi + C::kTile + c * kSlab, &tm_kl, bar(hReady + s), c * 64, kvh, ps.nb * 128, b);
             } else {
-              tma_load_4d(khi + c * kSlab, &tm_k, bar(hKFull + s), c * 64, kvh, ps.nb * 128, b);
+              tma_load_4d(khi + c * kSlab, &tm_k, bar(hReady + s), c * 64, kvh, ps.nb * 128, b);
             }
           }
           k_last = p;
+          // V(p): its stage is free once P V of pass p - 2 has completed, and
+          // by then the phase of pass p is open
+          if (p >= 2) {
+            if (!(ok = mbar_wait(bar(hVEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
+            mbar_expect_tx(bar(hReady + s), (uint32_t)C::kTile);
+          }
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(vdst + c * kSlab, &tm_v, bar(hReady + s), c * 64, kvh, ps.nb * 128, b);
+          v_last = p;
+          if (p + 2 >= npass) {
+            // no K(p + 2): pass p's phase gets the producer's arrival now
+            if (p < 2 && !(ok = mbar_wait(bar(hReady + s), 0u, abort_flag, args.dev_error))) break;
+            mbar_arrive(bar(hReady + s));
+          }
+        } else {
+          if (!(ok = mbar_wait(bar(hVEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
+          mbar_arrive_expect_tx(bar(hVFull + s), (uint32_t)C::kTile);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(vdst + c * kSlab, &tm_v, bar(hVFull + s), c * 64, kvh, ps.nb * 128, b);
+          v_last = p;
         }
-        if (!(ok = mbar_wait(bar(hVEmpty + s), ph ^ 1u, abort_flag, args.dev_error))) break;
-        mbar_arrive_expect_tx(bar(hVFull + s), (uint32_t)C::kTile);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sbase + C::kVOff + s * C::kTile + c * kSlab, &tm_v, bar(hVFull + s), c * 64, kvh,
-                      ps.nb * 128, b);
-        v_last = p;
       }
       if (!ok) {
-        // Let every copy already issued land before the CTA can exit.
+        // Let every copy already issued land before the CTA can exit.  (With
+        // pre-rotated keys a pass barrier also waits for softmax arrivals
+        // that an abort may never bring, so those waits end on their bound.)
         for (int p = max(0, k_last - kHStages + 1); p <= k_last; ++p)
-          h_drain_wait(bar(hKFull + (p & 1)), (uint32_t)(p >> 1) & 1u);
-        for (int p = max(0, v_last - kHStages + 1); p <= v_last; ++p)
-          h_drain_wait(bar(hVFull + (p & 1)), (uint32_t)(p >> 1) & 1u);
+          h_drain_wait(bar(hReady + (p & 1)), (uint32_t)(p >> 1) & 1u);
+        for (int p = max(0, v_last - kHStages + 1); p <= v_last; ++p) {
+          if constexpr (kRotK)
+            h_drain_wait(bar(hVFull + (p & 1)), (uint32_t)(p >> 1) & 1u);
+          else if (p >= 2)
+            h_drain_wait(bar(hReady + (p & 1)), (uint32_t)((p >> 1) + 1) & 1u);
+        }
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
@@ -341,19 +378,15 @@ __global__ void __launch_bounds__(kHThreads, 1)
       // passes with corrected (hi + lo) operands: the fused method's remote
       // passes come first; the single-kind calls use one operand kind
       const int n_hilo = kKind == kBifocal ? sc.n_rem : (kKind != kWindowBase ? npass : 0);
-      auto issue_s = [&](int p) -> bool {
-        const int s = p & 1;
-        const uint32_t ph = (uint32_t)(p >> 1) & 1u;
-        if (p == 0 || (q_switch && p == p_switch)) {
-          if (!mbar_wait(bar(hQReady), p == 0 ? 0u : 1u, abort_flag, args.dev_error)) return false;
-        }
-        if (!mbar_wait(bar(hKFull + s), ph, abort_flag, args.dev_error)) return false;
-        tc_fence_after();
+      // Score products of pass q into S buffer q % 2, then its commit (the
+      // softmax may read S; the key stage is free).
+      auto s_products = [&](int q) {
+        const int s = q & 1;
         const uint32_t d = tmem + (uint32_t)(128 * s);
         // descriptors of the stage's K_hi / K_lo tiles (k-step offsets are
         // added below as compile-time constants: one add per MMA)
         const uint64_t dkh = s == 0 ? dk_hi0 : dk_hi1;
-        if (p < n_hilo) {
+        if (q < n_hilo) {
           const uint64_t dkl = dkh + (uint64_t)(C::kTile >> 4);
           // Q_hi K_hi + Q_hi K_lo + Q_lo K_hi into one accumulator
 #pragma unroll
@@ -371,16 +404,11 @@ __global__ void __launch_bounds__(kHThreads, 1)
             mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_loc, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(hSFull + s));
-        if (q_switch && p == p_switch - 1) tc_commit(bar(hQEmpty));
-        return true;
+        if (q_switch && q == p_switch - 1) tc_commit(bar(hQEmpty));
       };
-      // O += P V once the softmax has written all of P.
-      auto issue_pv = [&](int p) -> bool {
+      // O += P V of pass p, then its commit (V stage free; O holds the pass).
+      auto pv_products = [&](int p) {
         const int s = p & 1;
-        const uint32_t ph = (uint32_t)(p >> 1) & 1u;
-        if (!mbar_wait(bar(hVFull + s), ph, abort_flag, args.dev_error)) return false;
-        if (!mbar_wait(bar(hPFull + s), ph, abort_flag, args.dev_error)) return false;
-        tc_fence_after();
         const uint64_t dv = s == 0 ? dv0 : dv1;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -390,15 +418,62 @@ __global__ void __launch_bounds__(kHThreads, 1)
                  (p > 0 || ks > 0) ? 1u : 0u);
         }
         tc_commit(bar(hVEmpty + s));
+      };
+      // the query operands of pass q (the first pass kind, or the base rows
+      // after the switch) must be in TMEM
+      auto wait_q = [&](int q) -> bool {
+        if (q == 0 || (q_switch && q == p_switch))
+          return mbar_wait(bar(hQReady), q == 0 ? 0u : 1u, abort_flag, args.dev_error);
         return true;
       };
       bool ok = true;
-      if (npass > 0) {
-        ok = issue_s(0);
-        if (ok && npass > 1) ok = issue_s(1);
+      if constexpr (!kRotK) {
+        // MMA order S(0) S(1) PV(0) S(2) PV(1) ...: one wait per pass, on the
+        // pass barrier that holds P(p), V(p) and K(p + 2).
+        for (int q = 0; q < 2 && q < npass && ok; ++q) {
+          ok = wait_q(q) && mbar_wait(bar(hReady + q), 0u, abort_flag, args.dev_error);
+          if (!ok) break;
+          tc_fence_after();
+          s_products(q);
+        }
         for (int p = 0; p < npass && ok; ++p) {
-          ok = issue_pv(p);
-          if (ok && p + 2 < npass) ok = issue_s(p + 2);
+          const int s = p & 1;
+          if (!(ok = mbar_wait(bar(hReady + s), (uint32_t)((p >> 1) + 1) & 1u, abort_flag, args.dev_error))) break;
+          tc_fence_after();
+          pv_products(p);
+          if (p + 2 < npass) {
+            if (q_switch && p + 2 == p_switch) {
+              if (!(ok = wait_q(p + 2))) break;
+              tc_fence_after();
+            }
+            s_products(p + 2);
+          }
+        }
+      } else {
+        auto issue_s = [&](int q) -> bool {
+          if (!wait_q(q)) return false;
+          if (!mbar_wait(bar(hReady + (q & 1)), (uint32_t)(q >> 1) & 1u, abort_flag, args.dev_error)) return false;
+          tc_fence_after();
+          s_products(q);
+          return true;
+        };
+        // O += P V once the softmax has written all of P.
+        auto issue_pv = [&](int p) -> bool {
+          const int s = p & 1;
+          const uint32_t ph = (uint32_t)(p >> 1) & 1u;
+          if (!mbar_wait(bar(hVFull + s), ph, abort_flag, args.dev_error)) return false;
+          if (!mbar_wait(bar(hPFull + s), ph, abort_flag, args.dev_error)) return false;
+          tc_fence_after();
+          pv_products(p);
+          return true;
+        };
+        if (npass > 0) {
+          ok = issue_s(0);
+          if (ok && npass > 1) ok = issue_s(1);
+          for (int p = 0; p < npass && ok; ++p) {
+            ok = issue_pv(p);
+            if (ok && p + 2 < npass) ok = issue_s(p + 2);
+          }
         }
       }
       // Every product issued must have completed before TMEM is released.
@@ -422,6 +497,11 @@ __global__ void __launch_bounds__(kHThreads, 1)
     float m_used = -INFINITY;
     float l_sum = 0.f;
     bool ok = true;
+    if constexpr (!kRotK) {
+      // phase 0 of both pass barriers (the first two passes) has no P
+      mbar_arrive(bar(hReady + 0));
+      mbar_arrive(bar(hReady + 1));
+    }
 
     for (int p = 0; p < npass; ++p) {
       const int s = p & 1;
@@ -545,7 +625,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(hPFull + s));
+        mbar_arrive(bar(kRotK ? hPFull + s : hReady + s));
       }
       {
         float a0, a1;
@@ -773,7 +853,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
             sts128(unit_addr(khi, U), src[4 * U], src[4 * U + 1], src[4 * U + 2], src[4 * U + 3]);
         }
         fence_proxy_async_smem();  // the tensor core reads these rows through the async proxy
-        mbar_arrive(bar(hKFull + s));
+        mbar_arrive(bar(hReady + s));
         if (q_switch && p == p_switch) {
           // The remote query operands have been read for the last time: put
           // the base rows in their place.
