@@ -380,8 +380,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
       const int n_hilo = kKind == kBifocal ? sc.n_rem : (kKind != kWindowBase ? npass : 0);
       // Score products of pass q into S buffer q % 2, then its commit (the
       // softmax may read S; the key stage is free).
-      auto s_products = [&](int q) {
-        const int s = q & 1;
+      auto s_products = [&](int q, int s) {  // s = q % 2, a constant at every call on the hot path
         const uint32_t d = tmem + (uint32_t)(128 * s);
         // descriptors of the stage's K_hi / K_lo tiles (k-step offsets are
         // added below as compile-time constants: one add per MMA)
@@ -407,8 +406,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
         if (q_switch && q == p_switch - 1) tc_commit(bar(hQEmpty));
       };
       // O += P V of pass p, then its commit (V stage free; O holds the pass).
-      auto pv_products = [&](int p) {
-        const int s = p & 1;
+      auto pv_products = [&](int p, int s) {  // s = p % 2
         const uint64_t dv = s == 0 ? dv0 : dv1;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -434,27 +432,37 @@ __global__ void __launch_bounds__(kHThreads, 1)
           ok = wait_q(q) && mbar_wait(bar(hReady + q), 0u, abort_flag, args.dev_error);
           if (!ok) break;
           tc_fence_after();
-          s_products(q);
+          s_products(q, q);
         }
-        for (int p = 0; p < npass && ok; ++p) {
-          const int s = p & 1;
-          if (!(ok = mbar_wait(bar(hReady + s), (uint32_t)((p >> 1) + 1) & 1u, abort_flag, args.dev_error))) break;
+        // One step per pass, unrolled by two so that each copy's parity (its
+        // S buffer, stage and barrier addresses) is a constant: every
+        // instruction between two products on this thread costs tensor time.
+        auto step = [&](int p, int s, uint32_t par) -> bool {
+          if (!mbar_wait(bar(hReady + s), par, abort_flag, args.dev_error)) return false;
           tc_fence_after();
-          pv_products(p);
+          pv_products(p, s);
           if (p + 2 < npass) {
             if (q_switch && p + 2 == p_switch) {
-              if (!(ok = wait_q(p + 2))) break;
+              if (!wait_q(p + 2)) return false;
               tc_fence_after();
             }
-            s_products(p + 2);
+            s_products(p + 2, s);
           }
+          return true;
+        };
+        uint32_t par = 1u;
+        int p = 0;
+        for (; p + 1 < npass && ok; p += 2) {
+          ok = step(p, 0, par) && step(p + 1, 1, par);
+          par ^= 1u;
         }
+        if (ok && p < npass) ok = step(p, 0, par);
       } else {
         auto issue_s = [&](int q) -> bool {
           if (!wait_q(q)) return false;
           if (!mbar_wait(bar(hReady + (q & 1)), (uint32_t)(q >> 1) & 1u, abort_flag, args.dev_error)) return false;
           tc_fence_after();
-          s_products(q);
+          s_products(q, q & 1);
           return true;
         };
         // O += P V once the softmax has written all of P.
@@ -464,7 +472,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
           if (!mbar_wait(bar(hVFull + s), ph, abort_flag, args.dev_error)) return false;
           if (!mbar_wait(bar(hPFull + s), ph, abort_flag, args.dev_error)) return false;
           tc_fence_after();
-          pv_products(p);
+          pv_products(p, s);
           return true;
         };
         if (npass > 0) {
