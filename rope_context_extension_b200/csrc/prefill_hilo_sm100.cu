@@ -17,9 +17,10 @@
 //     remote tile from global memory one tile ahead, rotates it in registers
 //     and writes hi / lo into shared memory in the 128-byte-swizzled K-major
 //     layout the tensor core reads (kRotK = true; no scratch, but measured
-//     about 3x slower on B200: the per-tile row loads, the second unrolled
-//     code region and the per-tile synchronisation cost more than the
-//     correction pass, which serves every query head of a KV head at once);
+//     3.7x slower at 128K on B200: the per-tile row loads, the second
+//     unrolled code region and the per-tile synchronisation cost more than
+//     the correction pass, which serves every query head of a KV head at
+//     once);
 //   * a remote score tile is S = Q_hi K_hi + Q_hi K_lo + Q_lo K_hi (fp32
 //     accumulate): a score's rounding error is about 2^-21 of |q| |k|
 //     instead of 2^-11 for one fp16 product (which is what a key of large norm
