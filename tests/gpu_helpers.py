@@ -101,3 +101,28 @@ def oracle_prefill_rows(q, k, v, rows, heads, p: jo.BifocalParams):
             qh = q[0, rows, h, :].double().numpy()
             out[h] = jo.attention_rows(qh, rows, kg, vg, p)
     return out
+
+
+def block_passes(L, w0, tile=128):
+    """(remote passes, local passes) of every 128-row query block: a key block
+    gets a remote pass if it holds a causal pair that is not local, a local
+    pass if it holds a local one (the oracle's is_local)."""
+    out = []
+    for a in range(-(-L // tile)):
+        i = np.arange(tile * a, min(tile * a + tile, L))
+        n_rem = n_loc = 0
+        for c in range(a + 1):
+            j = np.arange(tile * c, min(tile * c + tile, L))
+            causal = i[:, None] >= j[None, :]
+            loc = jo.is_local(i[:, None], j[None, :], w0)
+            n_loc += bool(np.any(causal & loc))
+            n_rem += bool(np.any(causal & ~loc))
+        out.append((n_rem, n_loc))
+    return out
+
+
+# (L, w0) with W = L / 2 (G 2): query blocks of one to five passes, the switch
+# from remote to local operands after pass 1, 2 or never, and blocks with only
+# local passes, i.e. the first passes of a block and its last ones, where the
+# prefill kernel's pipeline starts and drains
+SHORT_PASS_CASES = [(128, 0), (128, 64), (256, 0), (256, 100), (256, 200), (384, 0), (384, 150), (384, 260)]

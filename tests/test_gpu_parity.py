@@ -17,8 +17,8 @@ import torch
 from oracle import jetlong_oracle as jo
 from rope_context_extension_b200 import jetlong as jl
 from rope_context_extension_b200 import synthetic
-from tests.gpu_helpers import (LSE_MAX_ABS, PRECISIONS, assert_close, oracle_prefill_rows, prefill_workspace,
-                               run_decode, run_prefill, sample_rows)
+from tests.gpu_helpers import (LSE_MAX_ABS, PRECISIONS, SHORT_PASS_CASES, assert_close, oracle_prefill_rows,
+                               prefill_workspace, run_decode, run_prefill, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -68,6 +68,18 @@ def test_prefill_small_cases(B, L, Hq, Hkv, D, W, w0, mode, outl, prec):
     q, k, v = synthetic.prefill_inputs(B, L, Hq, Hkv, D, seed=L + w0, outlier_frac=outl)
     p = jo.BifocalParams(L=L, w0=w0, w_pretrained=W, base=10000.0, mode=mode)
     o, lse, err = run_prefill(q, k, v, w0=w0, W=W, base=10000.0, mode=mode, prec=prec)
+    assert err == 0
+    o_ref, lse_ref = jo.prefill_dense(q.float().numpy(), k.float().numpy(), v.float().numpy(), p)
+    assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"L{L} w0{w0} {prec}")
+
+
+@pytest.mark.parametrize("prec", ["default", "inkernel"])
+@pytest.mark.parametrize("L,w0", SHORT_PASS_CASES)
+def test_prefill_short_pass_sequences(L, w0, prec):
+    D = 128 if (L // 128 + w0) % 2 else 64
+    q, k, v = synthetic.prefill_inputs(1, L, 2, 1, D, seed=3 * L + w0, outlier_frac=0.01)
+    p = jo.BifocalParams(L=L, w0=w0, w_pretrained=L // 2, base=10000.0)
+    o, lse, err = run_prefill(q, k, v, w0=w0, W=L // 2, base=10000.0, prec=prec)
     assert err == 0
     o_ref, lse_ref = jo.prefill_dense(q.float().numpy(), k.float().numpy(), v.float().numpy(), p)
     assert_close(o.numpy(), o_ref, lse.numpy(), lse_ref, f"L{L} w0{w0} {prec}")

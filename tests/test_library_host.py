@@ -224,3 +224,18 @@ def test_wait_timeout_check_argument_errors(lib):
     assert lib.jl_wait_timeout_check(None, 0.1, None) == JL_ERR_INVALID_ARG
     assert lib.jl_wait_timeout_check(A, 0.0, None) == JL_ERR_INVALID_ARG
     assert lib.jl_wait_timeout_check(A, 11.0, None) == JL_ERR_INVALID_ARG
+
+
+def test_short_pass_sequences_cover_the_prefill_pipeline_edges():
+    # The GPU parity cases of tests.gpu_helpers.SHORT_PASS_CASES must contain
+    # query blocks whose pass sequences exercise the start and the end of the
+    # prefill kernel's pipeline: one remote pass, one local pass, a switch
+    # from remote to local operands after pass 1 and after pass 2, and two or
+    # three remote passes without a switch.
+    from tests.gpu_helpers import SHORT_PASS_CASES, block_passes
+    seen = {bp for L, w0 in SHORT_PASS_CASES for bp in block_passes(L, w0)}
+    for want in [(1, 0), (0, 1), (1, 1), (1, 2), (2, 2), (2, 0), (3, 0)]:
+        assert want in seen, want
+    # G 2 and w0 < L: every case runs the bifocal kernel, not the all-local one
+    for L, w0 in SHORT_PASS_CASES:
+        assert jo.group_size(L, L // 2) == 2 and w0 < L
