@@ -381,28 +381,40 @@ __global__ void __launch_bounds__(kHThreads, 1)
       const int n_hilo = kKind == kBifocal ? sc.n_rem : (kKind != kWindowBase ? npass : 0);
       // Score products of pass q into S buffer q % 2, then its commit (the
       // softmax may read S; the key stage is free).
-      auto s_products = [&](int q, int s) {  // s = q % 2, a constant at every call on the hot path
+      // The score products into S buffer s (= the pass's parity, a constant at
+      // every call on the hot path): remote passes Q_hi K_hi + Q_hi K_lo +
+      // Q_lo K_hi into one accumulator, local passes one bf16 product.
+      auto s_mmas_hilo = [&](int s) {
         const uint32_t d = tmem + (uint32_t)(128 * s);
         // descriptors of the stage's K_hi / K_lo tiles (k-step offsets are
         // added below as compile-time constants: one add per MMA)
         const uint64_t dkh = s == 0 ? dk_hi0 : dk_hi1;
-        if (q < n_hilo) {
-          const uint64_t dkl = dkh + (uint64_t)(C::kTile >> 4);
-          // Q_hi K_hi + Q_hi K_lo + Q_lo K_hi into one accumulator
+        const uint64_t dkl = dkh + (uint64_t)(C::kTile >> 4);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_rem, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_rem, ks > 0 ? 1u : 0u);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkl + kstep_off(ks), id_rem, 1u);
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkl + kstep_off(ks), id_rem, 1u);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(d, tmem + kColQB + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_rem, 1u);
-        } else {
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ts(d, tmem + kColQB + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_rem, 1u);
+      };
+      auto s_mmas_local = [&](int s) {
+        const uint32_t d = tmem + (uint32_t)(128 * s);
+        const uint64_t dkh = s == 0 ? dk_hi0 : dk_hi1;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_loc, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ts(d, tmem + kColQA + (uint32_t)(ks * 8), dkh + kstep_off(ks), id_loc, ks > 0 ? 1u : 0u);
+      };
+      // Score products of pass q with its commit (the softmax may read S; the
+      // key stage is free), and the query operands' release after the last
+      // remote pass.
+      auto s_products = [&](int q, int s) {
+        if (q < n_hilo)
+          s_mmas_hilo(s);
+        else
+          s_mmas_local(s);
         tc_commit(bar(hSFull + s));
         if (q_switch && q == p_switch - 1) tc_commit(bar(hQEmpty));
       };
@@ -435,13 +447,33 @@ __global__ void __launch_bounds__(kHThreads, 1)
           tc_fence_after();
           s_products(q, q);
         }
-        // One step per pass, unrolled by two so that each copy's parity (its
-        // S buffer, stage and barrier addresses) is a constant: every
-        // instruction between two products on this thread costs tensor time.
-        auto step = [&](int p, int s, uint32_t par) -> bool {
-          if (!mbar_wait(bar(hReady + s), par, abort_flag, args.dev_error)) return false;
+        // One step per pass: wait, P V(p), then S(p + 2).  The passes run in
+        // segments whose steps test nothing at run time (remote score
+        // products, local ones, none), with the one or two steps around the
+        // switch of query operands in between; each segment is unrolled by
+        // two so that each copy's parity (S buffer, stage, barrier addresses)
+        // is a constant.  Every instruction between two products on this
+        // thread costs tensor time.
+        auto pass_wait = [&](int p, int s) -> bool {
+          if (!mbar_wait(bar(hReady + s), (uint32_t)((p >> 1) + 1) & 1u, abort_flag, args.dev_error)) return false;
           tc_fence_after();
           pv_products(p, s);
+          return true;
+        };
+        auto step_hilo = [&](int p, int s) -> bool {
+          if (!pass_wait(p, s)) return false;
+          s_mmas_hilo(s);
+          tc_commit(bar(hSFull + s));
+          return true;
+        };
+        auto step_local = [&](int p, int s) -> bool {
+          if (!pass_wait(p, s)) return false;
+          s_mmas_local(s);
+          tc_commit(bar(hSFull + s));
+          return true;
+        };
+        auto step_any = [&](int p, int s) -> bool {
+          if (!pass_wait(p, s)) return false;
           if (p + 2 < npass) {
             if (q_switch && p + 2 == p_switch) {
               if (!wait_q(p + 2)) return false;
@@ -451,13 +483,24 @@ __global__ void __launch_bounds__(kHThreads, 1)
           }
           return true;
         };
-        uint32_t par = 1u;
-        int p = 0;
-        for (; p + 1 < npass && ok; p += 2) {
-          ok = step(p, 0, par) && step(p + 1, 1, par);
-          par ^= 1u;
-        }
-        if (ok && p < npass) ok = step(p, 0, par);
+        auto run = [&](int p0, int p1, auto&& body) {
+          int p = p0;
+          if (ok && p < p1 && (p & 1)) ok = body(p++, 1);
+          for (; p + 1 < p1 && ok; p += 2) ok = body(p, 0) && body(p + 1, 1);
+          if (ok && p < p1) ok = body(p, 0);
+        };
+        // iterations p issue S(p + 2) while p < npass - 2; it is remote while
+        // p + 2 < n_hilo; with a switch, p_switch = n_hilo and the steps that
+        // release the remote query operands (p_switch - 3) and wait for the
+        // base ones (p_switch - 2) test at run time
+        const int n_s = max(npass - 2, 0);
+        auto clampi = [&](int x) { return min(max(x, 0), n_s); };
+        const int a_end = clampi(q_switch ? n_hilo - 3 : n_hilo - 2);
+        const int b_end = clampi(q_switch ? n_hilo - 1 : n_hilo - 2);
+        run(0, a_end, step_hilo);
+        run(a_end, b_end, step_any);
+        run(b_end, n_s, step_local);
+        run(n_s, npass, pass_wait);
       } else {
         auto issue_s = [&](int q) -> bool {
           if (!wait_q(q)) return false;
