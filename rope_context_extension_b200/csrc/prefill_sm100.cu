@@ -242,9 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto kstep_off = [](int ks) -> uint64_t {
         return (uint64_t)(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
       };
-      auto issue_s = [&](int h, int p) -> bool {
-        const int s = p % kStages;
-        const uint32_t ph = (uint32_t)(p / kStages) & 1u;
+      auto issue_s = [&](int h, int p, int s) -> bool {  // s = p % 2
+        const uint32_t ph = (uint32_t)(p >> 1) & 1u;
         if (h == 0) {
           if (q_switch && p == sc.n_loc && !mbar_wait(bar(kQFull), 1, abort_flag, args.dev_error)) return false;
           if (!mbar_wait(bar(kKFull + s), ph, abort_flag, args.dev_error)) return false;
@@ -267,9 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_h += P V in two 64-key halves, each issued as soon as the softmax
       // has written that half of P, so the first half's product runs while
       // the second half's exponentials are taken.
-      auto issue_pv = [&](int h, int p) -> bool {
-        const int s = p % C::kVStages;
-        const uint32_t ph = (uint32_t)(p / C::kVStages) & 1u;
+      auto issue_pv = [&](int h, int p, int s) -> bool {  // s = p % 2
+        const uint32_t ph = (uint32_t)(p >> 1) & 1u;
         if (h == 0 && !mbar_wait(bar(kVFull + s), ph, abort_flag, args.dev_error)) return false;
         const uint64_t dv = s == 0 ? dv0 : dv1;
 #pragma unroll
@@ -292,13 +290,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (ok && npass > 0) {
         if (NH == 2) {
-          ok = issue_s(0, 0) && issue_s(1, 0) && issue_pv(0, 0);
-          for (int p = 1; p < npass && ok; ++p) {
-            ok = issue_s(0, p) && issue_pv(1, p - 1) && issue_s(1, p) && issue_pv(0, p);
-          }
-          if (ok) ok = issue_pv(1, npass - 1);
+          // unrolled by two passes so that each copy's stage parity is a constant
+          auto pass2 = [&](int p, int s) -> bool {
+            return issue_s(0, p, s) && issue_pv(1, p - 1, s ^ 1) && issue_s(1, p, s) && issue_pv(0, p, s);
+          };
+          ok = issue_s(0, 0, 0) && issue_s(1, 0, 0) && issue_pv(0, 0, 0);
+          int p = 1;
+          for (; p + 1 < npass && ok; p += 2) ok = pass2(p, 1) && pass2(p + 1, 0);
+          if (ok && p < npass) ok = pass2(p, 1);
+          if (ok) ok = issue_pv(1, npass - 1, (npass - 1) & 1);
         } else {
-          for (int p = 0; p < npass && ok; ++p) ok = issue_s(0, p) && issue_pv(0, p);
+          auto pass1 = [&](int p, int s) -> bool { return issue_s(0, p, s) && issue_pv(0, p, s); };
+          int p = 0;
+          for (; p + 1 < npass && ok; p += 2) ok = pass1(p, 0) && pass1(p + 1, 1);
+          if (ok && p < npass) ok = pass1(p, 0);
         }
       }
       // Every product issued must have completed before TMEM is released.
