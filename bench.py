@@ -213,15 +213,21 @@ class ClockSampler:
             self.thread.join(timeout=2)
         if self.handle is None and self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no NVML and no nvidia-smi"]}
-        t0 = self.window[0] if self.window[0] is not None else -math.inf
-        t1 = self.window[1] if self.window[1] is not None else math.inf
-        inside = [x for x in self.samples if t0 <= x[0] <= t1]
-        reasons = sorted(n for n, bit in self.REASONS.items() if any(x[3] & bit for x in inside))
-        return {"sm_mhz": statistics.median(x[1] for x in inside) if inside else None, "sm_max_mhz": self.smax,
+        return self.summarize(self.samples, self.window, self.smax,
+                              "nvml 20 ms" if self.handle is not None else "nvidia-smi 200 ms")
+
+    @classmethod
+    def summarize(cls, samples, window, smax, source):
+        """Clock summary of the samples (time, sm_mhz, power_w, reason bits)
+        taken inside window = [begin, end] (either may be None: unbounded)."""
+        t0 = window[0] if window[0] is not None else -math.inf
+        t1 = window[1] if window[1] is not None else math.inf
+        inside = [x for x in samples if t0 <= x[0] <= t1]
+        reasons = sorted(n for n, bit in cls.REASONS.items() if any(x[3] & bit for x in inside))
+        return {"sm_mhz": statistics.median(x[1] for x in inside) if inside else None, "sm_max_mhz": smax,
                 "sm_mhz_min": min(x[1] for x in inside) if inside else None,
                 "power_w_median": round(statistics.median(x[2] for x in inside), 1) if inside else None,
-                "reasons": reasons, "samples": len(inside),
-                "source": "nvml 20 ms" if self.handle is not None else "nvidia-smi 200 ms"}
+                "reasons": reasons, "samples": len(inside), "source": source}
 
 
 def dist_setup(n_gpus):

@@ -58,3 +58,30 @@ def test_our_arm_json_line_small():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
     dec = d["decode"]
     assert dec["roofline"]["bound"] == "hbm" and dec["value"] > 0
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_clock_summary_keeps_only_the_timed_window():
+    # (time, SM MHz, power W, clock-event reason bits); the timed region is
+    # [10, 20]: samples before and after it (idle clocks, a thermal event
+    # outside the region) must not count
+    cs = _bench_module().ClockSampler
+    samples = [(5.0, 1965.0, 200.0, 0x0), (9.9, 1965.0, 300.0, 0x40),
+               (10.0, 1500.0, 980.0, 0x4), (12.0, 1480.0, 990.0, 0x4), (15.0, 1520.0, 985.0, 0x4),
+               (20.0, 1510.0, 988.0, 0x4 | 0x8), (20.5, 1965.0, 250.0, 0x20)]
+    out = cs.summarize(samples, [10.0, 20.0], 1965.0, "test")
+    assert out["samples"] == 4
+    assert out["sm_mhz"] == 1505.0 and out["sm_mhz_min"] == 1480.0 and out["sm_max_mhz"] == 1965.0
+    assert out["power_w_median"] == 986.5
+    assert out["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    # no window: every sample counts; no sample inside: no clock
+    assert cs.summarize(samples, [None, None], 1965.0, "test")["samples"] == len(samples)
+    empty = cs.summarize(samples, [30.0, 40.0], 1965.0, "test")
+    assert empty["samples"] == 0 and empty["sm_mhz"] is None and empty["reasons"] == []
