@@ -14,9 +14,9 @@ step, summed over ranks, divided by the max-over-ranks device time of the
 prefill calls); the decode GB/s (K and V bytes read once) is reported beside
 it, and so are the other prefill paths (single fp16 product, key tiles
 corrected inside the kernel, the three-call inclusion-exclusion formulation,
-plain RoPE), the
-Qwen3-1.7B 64K and tiny workloads and the length / band sweep.  Inputs are
-larger than L2 (1 GiB Q, 4 GiB KV cache), so no flush runs between steps.
+plain RoPE), the Qwen3-1.7B 64K and tiny workloads, the length / band sweep,
+varlen decode, the new-token append and chunked prefill.  Inputs are larger
+than L2 (1 GiB Q, 4 GiB KV cache), so no flush runs between steps.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
 
@@ -557,6 +557,55 @@ def run_ours(args):
             del q2, k2, v2, o2, l2, w2
         others["length / band sweep (qwen3-4b shape, 1% x8 key outliers, decode B 1)"] = sweep
         del dws1
+
+        # varlen decode: one batch of the decode workload's cache whose
+        # sequences have lengths across the group sizes G = 1 .. 4 (the cache
+        # is read up to each sequence's own length)
+        Lm, Wd = Dc["L"], Dc["W"]
+        lens = [Lm // 8, Lm // 4, Lm // 4 + 1, 3 * Lm // 8, Lm // 2 + 1, 3 * Lm // 4, Lm, Lm][:Dc["B"]]
+        sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+        bsz = len(lens)
+        vms = time_calls(lambda: jl.jl_bifocal_decode_varlen(dq[:bsz], kc[:bsz], vc[:bsz], do[:bsz], dlse[:bsz], sl,
+                                                             max_len=Lm, w0=Dc["w0"], w_pretrained=Wd,
+                                                             rope_base=Dc["base"], workspace=dws, dev_error=err,
+                                                             stream=stream), 200)
+        vbytes = sum(2.0 * L_ * Dc["Hkv"] * Dc["D"] * 2.0 for L_ in lens)
+        hbm = load_peaks()[0]["hbm_gbs"]
+        others["varlen decode (qwen3-4b shape, mixed lengths)"] = {
+            "lengths": lens, "G": [jl.jl_group_size(L_, Wd) for L_ in lens], "ms": round(vms, 4),
+            "gbs": round(vbytes / (vms * 1e-3) / 1e9, 1), "frac": round(vbytes / (vms * 1e-3) / 1e9 / hbm, 4),
+            "tokens_per_s": round(bsz / (vms * 1e-3), 1)}
+        # the new-token append: rotate each sequence's new q and k at its
+        # position and write k, v into that cache row (the row after each
+        # length above, or the last row of a full cache; timed after the
+        # varlen call, which therefore read the cache unchanged)
+        qn = gen_on_device((bsz, Dc["Hq"], Dc["D"]), seed + 21, dev)
+        kn = gen_on_device((bsz, Dc["Hkv"], Dc["D"]), seed + 22, dev)
+        vn = gen_on_device((bsz, Dc["Hkv"], Dc["D"]), seed + 23, dev)
+        qo = torch.empty_like(qn)
+        pos = torch.tensor([min(L_, Lm - 1) for L_ in lens], dtype=torch.int32, device=dev)
+        ams = time_calls(lambda: jl.jl_rope_append(qn, kn, vn, pos, qo, kc[:bsz], vc[:bsz], rope_base=Dc["base"],
+                                                   dev_error=err, stream=stream), 1000)
+        others["new-token append (qwen3-4b shape, one token per sequence)"] = {
+            "B": bsz, "us": round(ams * 1e3, 2), "tokens_per_s": round(bsz / (ams * 1e-3), 1)}
+        del qn, kn, vn, qo
+        # chunked prefill: the prefill workload's last chunk of queries against
+        # its cache (the keys of every earlier position already there)
+        C_ = min(8192, P["L"] // 2)
+        off = P["L"] - C_
+        qc = q[:, off:].contiguous()
+        oc = torch.empty_like(qc)
+        lc = torch.empty(P["B"], P["Hq"], C_, dtype=torch.float32, device=dev)
+        wc = torch.empty(jl.jl_prefill_chunk_workspace_bytes(P["B"], off, C_, P["Hq"], P["Hkv"], P["D"]),
+                         dtype=torch.uint8, device=dev)
+        cms = time_calls(lambda: jl.jl_bifocal_prefill_chunk(qc, k, v, oc, lc, q_offset=off, w0=P["w0"],
+                                                             w_pretrained=P["W"], rope_base=P["base"], workspace=wc,
+                                                             dev_error=err, stream=stream), 5)
+        cflop = 4.0 * P["B"] * P["Hq"] * P["D"] * (C_ * off + C_ * (C_ + 1) / 2.0)
+        others["chunked prefill (qwen3-8b shape, last chunk of the prefill workload)"] = {
+            "q_offset": off, "chunk": C_, "ms": round(cms, 3), "tflops": round(cflop / (cms * 1e-3) / 1e12, 2),
+            "tokens_per_s": round(P["B"] * C_ / (cms * 1e-3), 1)}
+        del qc, oc, lc, wc
         if int(err.item()) != 0:
             raise RuntimeError(f"device error {int(err.item())} in the other workloads")
 
