@@ -606,6 +606,61 @@ def run_ours(args):
             "q_offset": off, "chunk": C_, "ms": round(cms, 3), "tflops": round(cflop / (cms * 1e-3) / 1e12, 2),
             "tokens_per_s": round(P["B"] * C_ / (cms * 1e-3), 1)}
         del qc, oc, lc, wc
+
+        # the multi-GPU decode layouts, one rank's share run alone on this GPU
+        # (the collective that follows is not included: the all-gather moves
+        # each rank's r x D outputs per head, a few KB): head sharding gives a
+        # rank Hkv / world KV heads of every sequence, sequence split gives it
+        # L / world keys of every sequence plus the combine of world partials
+        from rope_context_extension_b200 import multi_gpu as mg
+        layouts = []
+        def one_gpu():
+            return time_calls(lambda: jl.jl_bifocal_decode(dq, kc, vc, do, dlse, L=Dc["L"], w0=Dc["w0"],
+                                                           w_pretrained=Dc["W"], rope_base=Dc["base"], workspace=dws,
+                                                           dev_error=err, stream=stream), 100)
+        ms1 = one_gpu()
+        rank_ms = []
+        for world_ in (2, 4, 8):
+            entry = {"world": world_}
+            if Dc["Hkv"] % world_ == 0:
+                kb_, kn_, qb_, qn_ = mg.head_shard_slices(Dc["Hq"], Dc["Hkv"], 0, world_)
+                q_r, k_r, v_r = mg.take_heads(dq, qb_, qn_, dim=1), mg.take_heads(kc, kb_, kn_), mg.take_heads(vc, kb_, kn_)
+                o_r = torch.empty_like(q_r)
+                l_r = torch.empty(Dc["B"], qn_, dtype=torch.float32, device=dev)
+                ws_r = torch.zeros(jl.jl_decode_workspace_bytes(Dc["B"], Dc["L"], qn_, kn_, Dc["D"]), dtype=torch.uint8,
+                                   device=dev)
+                hms = time_calls(lambda: jl.jl_bifocal_decode(q_r, k_r, v_r, o_r, l_r, L=Dc["L"], w0=Dc["w0"],
+                                                              w_pretrained=Dc["W"], rope_base=Dc["base"], workspace=ws_r,
+                                                              dev_error=err, stream=stream), 100)
+                entry["head_shard_rank_ms"] = round(hms, 4)
+                rank_ms.append(("head_shard", entry, hms))
+                del q_r, k_r, v_r, o_r, l_r, ws_r
+            n_ = Dc["L"] // world_
+            k_s, v_s = kc[:, :n_].contiguous(), vc[:, :n_].contiguous()
+            o_s = torch.empty_like(dq)
+            l_s = torch.empty(Dc["B"], Dc["Hq"], dtype=torch.float32, device=dev)
+            ws_s = torch.zeros(jl.jl_decode_workspace_bytes(Dc["B"], n_, Dc["Hq"], Dc["Hkv"], Dc["D"]), dtype=torch.uint8,
+                               device=dev)
+            sms = time_calls(lambda: jl.jl_bifocal_decode_range(dq, k_s, v_s, o_s, l_s, key_offset=0, key_count=n_,
+                                                                total_len=Dc["L"], w0=Dc["w0"], w_pretrained=Dc["W"],
+                                                                rope_base=Dc["base"], workspace=ws_s, dev_error=err,
+                                                                stream=stream), 100)
+            o_p = o_s.unsqueeze(0).expand(world_, -1, -1, -1).contiguous()
+            l_p = l_s.unsqueeze(0).expand(world_, -1, -1).contiguous()
+            cms_ = time_calls(lambda: jl.jl_decode_combine(o_p, l_p, do, dlse, stream=stream), 100)
+            entry["sequence_split_rank_ms"] = round(sms, 4)
+            entry["sequence_split_combine_ms"] = round(cms_, 4)
+            rank_ms.append(("sequence_split", entry, sms + cms_))
+            layouts.append(entry)
+            del k_s, v_s, o_s, l_s, ws_s, o_p, l_p
+        # the one-GPU time before and after the shares (the clock under the
+        # power cap drifts between them); the lower one is the reference
+        ms1 = min(ms1, one_gpu())
+        for name_, entry, t_ in rank_ms:
+            entry[name_ + "_speedup_vs_one_gpu"] = round(ms1 / t_, 3)
+        others["multi-GPU decode layouts, one rank's share on one GPU (qwen3-4b shape, B 8)"] = {
+            "one_gpu_ms": round(ms1, 4), "ranks": layouts,
+            "note": "compute share of rank 0 alone; no collective and no second GPU"}
         if int(err.item()) != 0:
             raise RuntimeError(f"device error {int(err.item())} in the other workloads")
 
